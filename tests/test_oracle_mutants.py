@@ -1,0 +1,81 @@
+"""The pins must be sharp: each plausible mistake planted in a copy of the
+oracle's C source (compiled on the CPU into a temporary library) must make at
+least one pin fail.  Every mutant keeps its memory accesses in bounds."""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle as O
+from scaled_dot_product_14_b200 import inputs as I
+
+from test_oracle import _page1, _torch_ref, full, logical
+
+MUTANTS = {
+    "gqa_mapping_modulo": ("const int64_t g = h / n_rep;", "const int64_t g = h % Hkv;"),
+    "causal_top_left": ("if (j > i + (Lk - Lq)) sj = -INFINITY;", "if (j > i) sj = -INFINITY;"),
+    "causal_reversed": ("if (j > i + (Lk - Lq)) sj = -INFINITY;", "if (j < i + (Lk - Lq)) sj = -INFINITY;"),
+    "scale_dropped": ("double sj = scale * dot;", "double sj = dot;"),
+    "mask_subtracted": ("sj += oracle_load(mask, midx, dtype);", "sj -= oracle_load(mask, midx, dtype);"),
+    "bool_polarity": ("if (((const uint8_t*)mask)[midx] == 0) sj = -INFINITY;",
+                      "if (((const uint8_t*)mask)[midx] != 0) sj = -INFINITY;"),
+    "k_reversed_d": ("j * sk[2] + d * sk[3]", "j * sk[2] + (Dqk - 1 - d) * sk[3]"),
+    "no_normalise": ("for (int64_t e = 0; e < Dv; ++e) o[e] /= l;", ";"),
+    "mask_lq_index_dropped": ("i * (mask_st ? mask_st[2] : 0)", "0"),
+    "bf16_low_half": ("uint32_t bits = ((uint32_t)b) << 16;", "uint32_t bits = ((uint32_t)b) << 15;"),
+}
+
+
+def _pins_hold() -> bool:
+    """A compact set of pins; True if all hold for the currently loaded oracle."""
+    try:
+        import json
+        gold = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "mlx3585_linspace.json")))["printed"]
+        x, C, C_blhd, M, G = _page1(O)
+        if abs(np.abs(G - M).max() - gold["manual_vs_fused_max_diff"]) > 6e-8:
+            return False
+        if abs(np.abs(G - C_blhd).max() - gold["manual_vs_pytorch_fused_max_diff"]) > 6e-8:
+            return False
+        for mask in ["none", "additive", "bool", "causal"]:
+            c = I.make_case(77, 1, 4, 2, 6, 6, 64, dtype=I.BF16, mask=mask)
+            if c.mask_kind == I.MASK_BOOL:
+                c.mask.reshape(c.Lq, c.Lk)[:, 0] = 1
+            if np.abs(full(O, c) - _torch_ref(c)).max() > 1e-12:
+                return False
+        # causal with Lq != Lk: the query chunk [3, 4) of a Lq = 4 problem
+        c = I.make_case(78, 1, 2, 2, 4, 9, 64, dtype=I.F32, mask="causal")
+        last = full(O, c)[:, :, 3:4]
+        from test_oracle import with_values
+        sub = I.make_case(78, 1, 2, 2, 1, 9, 64, dtype=I.F32, mask="causal")
+        sub = with_values(sub, q=logical(c, "q")[:, :, 3:4], k=logical(c, "k"), v=logical(c, "v"))
+        if np.abs(full(O, sub) - last).max() > 1e-12:
+            return False
+        return True
+    except ValueError:
+        return False
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(tmp_path, oracle_mod, name):
+    src = open(os.path.join(os.path.dirname(O.__file__), "sdpa_oracle.c")).read()
+    old, new = MUTANTS[name]
+    assert src.count(old) == 1, name
+    path = tmp_path / "mut.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / "mut.so"
+    subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-o", str(so), str(path), "-lm"])
+    saved = O._load()
+    lib = ctypes.CDLL(str(so))
+    lib.oracle_sdpa_rows.restype = saved.oracle_sdpa_rows.restype
+    lib.oracle_sdpa_rows.argtypes = saved.oracle_sdpa_rows.argtypes
+    O._lib = lib
+    try:
+        assert not _pins_hold(), f"mutant {name} slipped through every pin"
+    finally:
+        O._lib = saved
+
+
+def test_unmutated_oracle_passes_the_same_pins(oracle_mod):
+    assert _pins_hold()

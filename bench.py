@@ -1,0 +1,473 @@
+#!/usr/bin/env python
+"""Benchmark of the fused SDPA forward on B200.
+
+Headline workload (one step = one decode call through the C ABI):
+  decode ("vector" path of MLX issue #3885): bf16, B=1, qL=1, kL=4096,
+  Hq=32, Hkv=8 (GQA 4), D=256, additive mask [1,1,1,kL] U(-1,0) with the last
+  10% of keys -inf; Q/K/V ~ N(0,1) seeded.
+Metric: decode KV GB/s = algorithmic bytes (K+V+Q+O footprint) / time; the
+prefill TFLOP/s of the head-dim-72 and head-dim-512 prefill workloads are
+reported alongside in "prefill".
+
+Timing: W warm-up steps, then K steps bracketed by a barrier and
+torch.cuda.synchronize() on both sides, CUDA events on the launching stream,
+max over ranks.  The K/V cache rotates over enough copies to exceed the
+126 MB L2, so every step reads K and V from HBM.  The steps are replayed from
+a CUDA graph (the decode call is a few microseconds; eager launches would time
+the host).  Multi-GPU: every rank runs the same per-GPU problem on its own
+copy (the (batch, KV-head) units are independent: no data-path collective),
+so scaling is weak and the value is the sum over ranks.
+
+``--impl reference`` times the float64 CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SDPA prefill TFLOP/s & decode KV GB/s on 1 B200, as fraction of roofline"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- workloads
+def decode_workload(kL=4096):
+    return dict(name=f"decode bf16 B=1 qL=1 kL={kL} Hq=32 Hkv=8 D=256 additive mask [1,1,1,kL] (last 10% -inf)",
+                seed=1001, B=1, Hq=32, Hkv=8, Lq=1, Lk=kL, Dqk=256, Dv=256, dtype="bf16", mask="decode_additive",
+                layout="bhld")
+
+
+PREFILL_WORKLOADS = [
+    dict(name="prefill bf16 B=1 H=16 L=8192 D=72 no mask [B,L,H,D]", seed=1003, B=1, Hq=16, Hkv=16, Lq=8192,
+         Lk=8192, Dqk=72, Dv=72, dtype="bf16", mask="none", layout="blhd"),
+    dict(name="prefill bf16 B=1 Hq=32 Hkv=4 L=4096 D=512 causal", seed=1002, B=1, Hq=32, Hkv=4, Lq=4096, Lk=4096,
+         Dqk=512, Dv=512, dtype="bf16", mask="causal", layout="bhld"),
+]
+
+
+def decode_bytes(w):
+    """Algorithmic bytes of one decode call: K+V read once, Q read, O written."""
+    e = 2 if w["dtype"] in ("bf16", "f16") else 4
+    kv = w["B"] * w["Hkv"] * w["Lk"] * (w["Dqk"] + w["Dv"])
+    qo = w["B"] * w["Hq"] * w["Lq"] * (w["Dqk"] + w["Dv"])
+    return e * (kv + qo)
+
+
+def prefill_flops(w):
+    f = 2.0 * w["B"] * w["Hq"] * w["Lq"] * w["Lk"] * (w["Dqk"] + w["Dv"])
+    return f / 2 if w["mask"] == "causal" else f
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "scaled_dot_product_14_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(key, files):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(key)
+    if not d or d.get("source_sha") != kernel_source_hash(files):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms while active."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        busy = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in busy:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in busy), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(busy), "power_w_max": max(r["power"] for r in rows)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- our arm
+def device_case(w, rank):
+    import torch
+    from scaled_dot_product_14_b200 import inputs as I
+    c = I.make_case(w["seed"] + 17 * rank, w["B"], w["Hq"], w["Hkv"], w["Lq"], w["Lk"], w["Dqk"], w["Dv"],
+                    dtype=I.DTYPE_BY_NAME[w["dtype"]], mask=w["mask"], layout=w["layout"])
+
+    def dev(a, is_mask=False):
+        if is_mask and c.mask_kind == I.MASK_BOOL:
+            return torch.from_numpy(a).cuda()
+        if c.dtype == I.F32:
+            return torch.from_numpy(a).cuda()
+        tdt = torch.bfloat16 if c.dtype == I.BF16 else torch.float16
+        return torch.from_numpy(a.view(np.int16)).view(tdt).cuda()
+
+    t = dict(q=dev(c.q), k=dev(c.k), v=dev(c.v), mask=None if c.mask is None else dev(c.mask, True))
+    return c, t
+
+
+def call(S, c, t, k, v, out, stream):
+    st = S.sdpa_forward(t["q"].data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), c.B, c.Hq, c.Hkv, c.Lq, c.Lk,
+                        c.Dqk, c.Dv, c.all_strides16, c.scale, c.mask_kind,
+                        None if t["mask"] is None else t["mask"].data_ptr(),
+                        None if t["mask"] is None else c.mask_strides, c.dtype, stream)
+    if st != 0:
+        raise S.SdpaError(st)
+
+
+def run_ours(args, peaks):
+    import torch
+    import scaled_dot_product_14_b200 as S
+    from scaled_dot_product_14_b200 import build
+    world, rank, local = dist_setup(args.gpus)
+    if rank == 0 and not os.path.exists(S.LIB_PATH):
+        build.build()
+    barrier(world)
+
+    w = decode_workload(args.kl)
+    c, t = device_case(w, rank)
+    bytes_per_step = decode_bytes(w)
+    kv_bytes = t["k"].numel() * 2 + t["v"].numel() * 2
+    copies = max(2, math.ceil(2 * L2_BYTES / kv_bytes))
+    ks = [t["k"]] + [t["k"].clone() for _ in range(copies - 1)]
+    vs = [t["v"]] + [t["v"].clone() for _ in range(copies - 1)]
+    out = torch.empty(c.B * c.Hq * c.Lq * c.Dv, dtype=t["q"].dtype, device="cuda")
+    stream = torch.cuda.Stream()
+    sp = stream.cuda_stream
+
+    with torch.cuda.stream(stream):
+        call(S, c, t, ks[0], vs[0], out, sp)          # allocates the split-K workspace before capture
+    torch.cuda.synchronize()
+    launches_per_step = S.sdpa_last_launch_count()
+
+    # a graph holding one step per K/V copy; replays cycle through the copies
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(copies):
+            call(S, c, t, ks[i], vs[i], out, sp)
+    torch.cuda.synchronize()
+    steps = args.steps
+    reps = max(1, math.ceil(steps / copies))
+    steps_run = reps * copies
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    for _ in range(max(args.warmup, 3)):
+        with torch.cuda.stream(stream):
+            call(S, c, t, ks[0], vs[0], out, sp)
+    # untimed soak so that clock samples see the GPU under this load
+    soak_end = time.time() + args.soak
+    while time.time() < soak_end:
+        graph.replay()
+        stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms, world)
+    ms_per_step = ms / steps_run
+    value = world * bytes_per_step * steps_run / (ms * 1e-3) / 1e9
+
+    # dominant kernel alone: event-bracketed launches on the same stream (eager, same copies)
+    S.sdpa_profile_enable(True)
+    S.sdpa_profile_collect()
+    for r in range(max(4, 2 * copies)):
+        with torch.cuda.stream(stream):
+            call(S, c, t, ks[r % copies], vs[r % copies], out, sp)
+    torch.cuda.synchronize()
+    prof = S.sdpa_profile_collect()
+    S.sdpa_profile_enable(False)
+    n_dec, ms_dec = prof["decode_mma"]
+    n_cmb, ms_cmb = prof["combine"]
+    dec_us = 1e3 * ms_dec / max(n_dec, 1)
+    achieved = bytes_per_step / (dec_us * 1e-6) / 1e9
+    traffic = ncu_traffic(f"decode_mma kL={args.kl}", ["decode_mma.cu", "common.cuh", "kernels.h"])
+    roof = {"bound": "hbm", "kernel": "decode_mma_kernel", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic, "algorithmic_bytes_per_launch": bytes_per_step,
+            "kernel_us": round(dec_us, 3), "combine_us": round(1e3 * ms_cmb / max(n_cmb, 1), 3),
+            "peak_source": f"{peaks['source']} hbm_gbs (copy, burst)"}
+
+    result = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": steps_run,
+              "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
+              "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+              "config": {"workload": w["name"], "kv_copies_rotated": copies,
+                         "l2": f"inputs larger than L2: {copies} rotating K/V copies "
+                               f"({copies * kv_bytes / 2**20:.0f} MiB > 126 MB L2)",
+                         "launch": "CUDA graph replay of the C-ABI calls", "soak_s": args.soak,
+                         "parallelism": f"replicas x{world} (no collective)"},
+               "roofline": roof, "clocks": clk, "gpu_launches": launches_per_step * steps_run}
+
+    if not args.no_e2e:
+        result["e2e"] = e2e(S, c, t, out, stream, args, world)
+    if not args.no_prefill:
+        result["prefill"] = prefill_leg(S, stream, peaks, rank, args)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del graph
+        dist.destroy_process_group()
+
+
+def e2e(S, c, t, out, stream, args, world):
+    """Same metric through the C ABI from pinned host buffers: H2D of the step's
+    inputs, the call, D2H of the output, all inside the timed region."""
+    import torch
+    host = {k: v.cpu().pin_memory() for k, v in t.items() if v is not None}
+    dev = {k: torch.empty_like(v) for k, v in t.items() if v is not None}
+    host_out = torch.empty(out.numel(), dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out.numel() * out.element_size()
+    n = max(3, min(args.steps, 50))
+
+    def step():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        td = dict(dev)
+        td.setdefault("mask", None)
+        call(S, c, td, dev["k"], dev["v"], out, stream.cuda_stream)
+        host_out.copy_(out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    val = world * decode_bytes(decode_workload(args.kl)) * n / (ms * 1e-3) / 1e9
+    return {"value": round(val, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": n, "ms_per_step": round(ms / n, 4)}
+
+
+def prefill_leg(S, stream, peaks, rank, args):
+    import torch
+    res = []
+    for w in PREFILL_WORKLOADS:
+        c, t = device_case(w, rank)
+        out = torch.empty(c.B * c.Hq * c.Lq * c.Dv, dtype=t["q"].dtype, device="cuda")
+        sp = stream.cuda_stream
+        with torch.cuda.stream(stream):
+            call(S, c, t, t["k"], t["v"], out, sp)
+            torch.cuda.synchronize()
+            first = time.time()
+            call(S, c, t, t["k"], t["v"], out, sp)
+            torch.cuda.synchronize()
+            one = time.time() - first
+            n = int(max(3, min(20, 2.0 / max(one, 1e-4))))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                call(S, c, t, t["k"], t["v"], out, sp)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / n
+        fl = prefill_flops(w)
+        tf = fl / (ms * 1e-3) / 1e12
+        cnt = S.sdpa_get_counters()
+        res.append({"workload": w["name"], "ms": round(ms, 4), "tflops": round(tf, 2),
+                    "algorithmic_flops": fl, "peak_tflops": peaks["bf16_tflops"],
+                    "frac": round(tf / peaks["bf16_tflops"], 4), "bound": "tensor",
+                    "kernel": "prefill_tcgen05" if cnt["prefill_tcgen05_launches"] else "prefill_ffma",
+                    "iters": n})
+        del t, out
+        torch.cuda.empty_cache()
+    return res
+
+
+def cpu_baseline(w, seconds):
+    """The float64 oracle as it stands on this host's cores, on full decode steps."""
+    import oracle
+    from scaled_dot_product_14_b200 import inputs as I
+    oracle.build()
+    c = I.make_case(w["seed"], w["B"], w["Hq"], w["Hkv"], w["Lq"], w["Lk"], w["Dqk"], w["Dv"],
+                    dtype=I.DTYPE_BY_NAME[w["dtype"]], mask=w["mask"], layout=w["layout"])
+    threads = os.cpu_count() or 1
+    n, t0 = 0, time.time()
+    while True:
+        oracle.sdpa_rows(c.q, c.k, c.v, B=c.B, Hq=c.Hq, Hkv=c.Hkv, Lq=c.Lq, Lk=c.Lk, Dqk=c.Dqk, Dv=c.Dv,
+                         strides=c.strides, scale=c.scale, dtype=c.dtype, mask_kind=c.mask_kind, mask=c.mask,
+                         mask_strides=c.mask_strides, threads=threads)
+        n += 1
+        if time.time() - t0 >= seconds or n >= 1000:
+            break
+    el = time.time() - t0
+    return {"value": round(decode_bytes(w) * n / el / 1e9, 4), "unit": "GB/s", "cores": min(threads, c.B * c.Hq),
+            "kind": "oracle", "sample": f"{n} full decode steps ({c.B * c.Hq} query rows x {c.Lk} keys each) "
+                                        f"in {el:.1f} s; rows split over host threads"}
+
+
+# ----------------------------------------------------------------------------- reference arm (the oracle)
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from scaled_dot_product_14_b200 import inputs as I
+    oracle.build()
+    w = decode_workload(args.kl)
+    c = I.make_case(w["seed"], w["B"], w["Hq"], w["Hkv"], w["Lq"], w["Lk"], w["Dqk"], w["Dv"],
+                    dtype=I.DTYPE_BY_NAME[w["dtype"]], mask=w["mask"], layout=w["layout"])
+    threads = os.cpu_count() or 1
+
+    def step():
+        oracle.sdpa_rows(c.q, c.k, c.v, B=c.B, Hq=c.Hq, Hkv=c.Hkv, Lq=c.Lq, Lk=c.Lk, Dqk=c.Dqk, Dv=c.Dv,
+                         strides=c.strides, scale=c.scale, dtype=c.dtype, mask_kind=c.mask_kind, mask=c.mask,
+                         mask_strides=c.mask_strides, threads=threads)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    t0 = time.time()
+    for _ in range(args.steps):
+        step()
+    el = time.time() - t0
+    val = decode_bytes(w) * args.steps / el / 1e9
+    cores = min(threads, c.B * c.Hq)
+    print(json.dumps({"metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": world,
+                      "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * el / args.steps, 3),
+                      "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                      "data": "synthetic", "impl": "reference",
+                      "config": {"workload": w["name"], "parallelism": "host threads (oracle)"},
+                      "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                       "sample": f"each step = one full decode call ({c.B * c.Hq} rows x {c.Lk} keys)"},
+                      "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                              "d2h_bytes_per_step": 0}}), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--kl", type=int, default=4096, help="decode key length (1024 or 4096 on the pages)")
+    ap.add_argument("--soak", type=float, default=1.0, help="untimed seconds under load before timing")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args, load_peaks())
+
+
+if __name__ == "__main__":
+    main()

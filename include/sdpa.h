@@ -1,0 +1,206 @@
+/*
+ * sdpa.h -- C ABI of the B200 (sm_100a) fused scaled-dot-product attention
+ * forward pass.
+ *
+ * Operation (per batch b, query head h, query row i):
+ *
+ *     out[b,h,i,:] = softmax_j( scale * q[b,h,i,:] . k[b,g,j,:] + mask[b,h,i,j] ) . v[b,g,j,:]
+ *
+ *   - the definition is the fixed composite of MLX issue #3585
+ *     ("mx.fast.scaled_dot_product_attention produces incorrect attention
+ *     scores (MLX 0.31.2)"), section "Reproduction": scores = q k^T * scale,
+ *     softmax along the key axis, times v;
+ *   - GQA: g = h / (Hq / Hkv), the contiguous grouping [B, n_kv, n_rep, qL, kL]
+ *     of MLX issue #3885 ("Metal SDPA: no fused path for head_dim=512"),
+ *     section "Measured impact";
+ *   - path split: Lq <= 8 runs the decode ("vector") path, Lq > 8 the prefill
+ *     ("full") path, as in that issue's section "Current routing";
+ *   - head dims: Dqk in {64, 72, 80, 96, 128, 192, 256, 512} with Dv == Dqk,
+ *     plus (Dqk, Dv) = (192, 128) (same section; head dim 72 from MLX PR #4330
+ *     "Support head dimension 72 in Metal full attention");
+ *   - masks: none, additive, boolean, causal (MLX PR #4330, "Proposed changes").
+ *
+ * Layout is never inferred from a tensor's shape: every tensor is passed as a
+ * base pointer plus explicit (b, h, l, d) element strides, so [B,L,H,D] and
+ * [B,H,L,D] buffers (or any other strided view) are described exactly.  The
+ * layout misread of MLX issue #3585, section "Root cause analysis", cannot
+ * happen through this interface.
+ *
+ * Readings where the pages are silent:
+ *   - additive mask is added after scaling; -inf entries remove a key;
+ *   - boolean mask: nonzero = attend, zero = removed;
+ *   - causal with Lq != Lk is aligned bottom-right: key j is visible to query
+ *     i iff j <= i + (Lk - Lq);
+ *   - a query row with no visible key yields zeros (never NaN).
+ *
+ * Threading: the functions are thread-safe.  Execution is asynchronous on the
+ * caller's stream; validation is synchronous and happens before any launch.
+ * There is no fallback path of any kind: a case the kernels do not cover is
+ * rejected with an error status and nothing is launched.
+ */
+#ifndef SDPA_B200_SDPA_H
+#define SDPA_B200_SDPA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element types of q, k, v, out (and of an additive mask). */
+typedef enum {
+    SDPA_F32 = 0,   /* IEEE binary32; computed in true fp32 (no TF32, no fp16 rounding) */
+    SDPA_F16 = 1,   /* IEEE binary16 storage, fp32 accumulation */
+    SDPA_BF16 = 2   /* bfloat16 storage, fp32 accumulation */
+} sdpa_dtype;
+
+typedef enum {
+    SDPA_MASK_NONE = 0,      /* mask must be NULL */
+    SDPA_MASK_ADDITIVE = 1,  /* mask: same element type as q, added to scale*q.k */
+    SDPA_MASK_BOOL = 2,      /* mask: uint8, nonzero = attend */
+    SDPA_MASK_CAUSAL = 3     /* mask must be NULL; bottom-right aligned */
+} sdpa_mask_kind;
+
+typedef enum {
+    SDPA_OK = 0,
+    SDPA_ERR_INVALID_ARG = 1,         /* negative size, Hq % Hkv != 0, bad enum, non-finite scale */
+    SDPA_ERR_UNSUPPORTED_DIM = 2,     /* (Dqk, Dv) not in the supported set */
+    SDPA_ERR_UNSUPPORTED_STRIDE = 3,  /* d-stride != 1, negative stride, or a stride that is not a
+                                         multiple of 16 bytes */
+    SDPA_ERR_MISALIGNED = 4,          /* a base pointer not 16-byte aligned */
+    SDPA_ERR_LAUNCH_CONFIG = 5,       /* the launch shape exceeds a device limit (grid size,
+                                         shared memory); nothing was launched */
+    SDPA_ERR_CUDA = 6,                /* a CUDA runtime call failed (see sdpa_last_cuda_error) */
+    SDPA_ERR_TIMEOUT = 7,             /* a bounded in-kernel wait ran out (debug check only) */
+    SDPA_ERR_NO_MEMORY = 8,           /* the split-K workspace could not be allocated */
+    SDPA_ERR_NULL_POINTER = 9,        /* q, k, v or out is NULL (with a non-empty problem), or the
+                                         mask pointer does not match mask_kind */
+    SDPA_ERR_TOO_LARGE = 10           /* a size exceeds the kernels' index range */
+} sdpa_status;
+
+typedef enum {
+    SDPA_PATH_NONE = 0,     /* empty problem: nothing to launch */
+    SDPA_PATH_PREFILL = 1,  /* Lq > 8: tiled flash kernel (tcgen05 for fp16/bf16, FFMA for fp32) */
+    SDPA_PATH_DECODE = 2    /* Lq <= 8: split-K kernel plus log-sum-exp combine */
+} sdpa_path;
+
+/*
+ * sdpa_forward -- out = softmax(scale * q k^T + mask) v.
+ *
+ * q    : device pointer, element (b,h,i,d) at q + b*s[0] + h*s[1] + i*s[2] + d*s[3]   (h < Hq,  i < Lq, d < Dqk)
+ * k    : device pointer, element (b,g,j,d) at k + b*s[4] + g*s[5] + j*s[6] + d*s[7]   (g < Hkv, j < Lk, d < Dqk)
+ * v    : device pointer, element (b,g,j,e) at v + b*s[8] + g*s[9] + j*s[10] + e*s[11] (g < Hkv, j < Lk, e < Dv)
+ * out  : device pointer, element (b,h,i,e) at out + b*s[12] + h*s[13] + i*s[14] + e*s[15]
+ *        (the only memory the call writes besides the library's own workspace)
+ * strides : 16 element strides (not bytes).  Requirements: every d-stride
+ *        (s[3], s[7], s[11], s[15]) is 1; every other stride is >= 0 and, times
+ *        the element size, a multiple of 16 bytes (a stride whose dimension has
+ *        extent 1 is not checked).
+ * scale: multiplies q.k before the mask is added (usually Dqk^-0.5).
+ * mask_kind / mask / mask_strides:
+ *        ADDITIVE: mask element (b,h,i,j) at mask + b*m[0] + h*m[1] + i*m[2] + j*m[3],
+ *                  element type = dtype; strides in elements, 0 broadcasts.
+ *        BOOL:     same indexing, uint8 elements.
+ *        NONE / CAUSAL: mask and mask_strides must be NULL.
+ * dtype : sdpa_dtype of q, k, v, out.
+ * stream: a cudaStream_t (NULL = the legacy default stream).
+ *
+ * Requirements: Hq % Hkv == 0; (Dqk, Dv) supported; base pointers 16-byte
+ * aligned.  out must not overlap q, k, v or mask.
+ * Empty problems (B, Hq or Lq == 0) return SDPA_OK without launching; Lk == 0
+ * writes zeros to out.
+ * Ownership: all pointers are the caller's.  The decode path uses a split-K
+ * workspace the library allocates on first use per (device, stream), keeps,
+ * and frees in sdpa_shutdown(); two calls on the same stream share it safely
+ * because the stream orders them.
+ * Returns an sdpa_status.  On any status other than SDPA_OK and SDPA_ERR_CUDA
+ * nothing was launched.
+ */
+int sdpa_forward(const void* q, const void* k, const void* v, void* out,
+                 int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk,
+                 int64_t Dqk, int64_t Dv, const int64_t strides[16], float scale,
+                 int mask_kind, const void* mask, const int64_t mask_strides[4],
+                 int dtype, void* stream);
+
+/*
+ * sdpa_supported -- the same validation sdpa_forward runs, without pointers
+ * and without launching.  Writes the path that would run (sdpa_path) to
+ * *path_out when path_out is not NULL.  Returns an sdpa_status; SDPA_OK means
+ * sdpa_forward would accept these sizes and strides (given aligned pointers).
+ */
+int sdpa_supported(int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk,
+                   int64_t Dqk, int64_t Dv, const int64_t strides[16], int mask_kind,
+                   const int64_t mask_strides[4], int dtype, int* path_out);
+
+/* Static text for a status code. */
+const char* sdpa_error_string(int status);
+
+/* Text of the last CUDA error seen by this thread's sdpa_forward ("" if none). */
+const char* sdpa_last_cuda_error(void);
+
+/*
+ * Call counters (process-wide).  Invariant:
+ *   calls == prefill_calls + decode_calls + empty_calls + rejected_calls.
+ * The kernel counters say which kernel family served each call.
+ */
+typedef struct {
+    uint64_t calls;
+    uint64_t prefill_calls;
+    uint64_t decode_calls;
+    uint64_t empty_calls;
+    uint64_t rejected_calls;
+    uint64_t prefill_tcgen05_launches;  /* fp16/bf16 prefill on tcgen05 tensor cores */
+    uint64_t prefill_ffma_launches;     /* fp32 prefill on CUDA cores */
+    uint64_t decode_mma_launches;       /* fp16/bf16 split-K decode */
+    uint64_t decode_ffma_launches;      /* fp32 split-K decode */
+    uint64_t combine_launches;          /* log-sum-exp combine of split-K partials */
+} sdpa_counters;
+
+void sdpa_get_counters(sdpa_counters* out);
+void sdpa_reset_counters(void);
+
+/*
+ * Kernel launches the most recent successful sdpa_forward on this thread
+ * made (1 or 2).  Lets a caller count launches without a profiler.
+ */
+int sdpa_last_launch_count(void);
+
+/*
+ * Reads and clears the device-side error flag that bounded in-kernel waits
+ * set when they give up (0 = none).  Synchronises the stream.  Returns an
+ * sdpa_status: SDPA_ERR_TIMEOUT if the flag was set.
+ */
+int sdpa_check_device_error(void* stream, int* code_out);
+
+/*
+ * Optional per-kernel timing with CUDA events (off by default).  While
+ * enabled, sdpa_forward brackets every kernel it launches with two events
+ * recorded on the call's stream.  sdpa_profile_collect waits for those events,
+ * adds their elapsed times per kernel family into launches[] / total_ms[]
+ * (arrays of SDPA_KERNEL_FAMILIES entries, indexed by sdpa_kernel_family),
+ * and forgets them.  Nothing else changes: the same kernels run.
+ */
+typedef enum {
+    SDPA_KERNEL_PREFILL_TCGEN05 = 0,
+    SDPA_KERNEL_PREFILL_FFMA = 1,
+    SDPA_KERNEL_DECODE_MMA = 2,
+    SDPA_KERNEL_DECODE_FFMA = 3,
+    SDPA_KERNEL_COMBINE = 4,
+    SDPA_KERNEL_ZERO_FILL = 5,
+    SDPA_KERNEL_FAMILIES = 6
+} sdpa_kernel_family;
+
+int sdpa_profile_enable(int on);
+int sdpa_profile_collect(uint64_t launches[SDPA_KERNEL_FAMILIES], double total_ms[SDPA_KERNEL_FAMILIES]);
+
+/* Frees every cached workspace.  Call with no sdpa work in flight. */
+int sdpa_shutdown(void);
+
+/* ABI version of this header (increases on incompatible change). */
+int sdpa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDPA_B200_SDPA_H */

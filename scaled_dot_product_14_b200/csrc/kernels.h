@@ -1,0 +1,86 @@
+// kernels.h -- internal interface between the host dispatcher (api.cu) and the
+// kernel translation units.  Not part of the public ABI (include/sdpa.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sdpa {
+
+// Each kernel translation unit holds its own copy of this flag (internal
+// linkage, no relocatable device code).  A bounded wait that gives up writes a
+// nonzero code here; the host reads and clears it through the unit's
+// take_device_error_* function.
+static __device__ int g_sdpa_device_error = 0;
+
+enum DeviceErrorCode : int {
+    kErrNone = 0,
+    kErrWaitTmaLoad = 1,     // producer-side data never arrived
+    kErrWaitMma = 2,         // an MMA completion never arrived
+    kErrWaitSoftmax = 3,     // the softmax warps never released a buffer
+    kErrWaitSlot = 4,        // a ring slot was never freed
+};
+
+// Everything a kernel needs to address one attention problem.  Strides are in
+// elements; the dispatcher has already validated them.
+struct AttnParams {
+    const void* q;
+    const void* k;
+    const void* v;
+    void* out;
+    const void* mask;
+    int64_t B, Hq, Hkv, Lq, Lk, Dqk, Dv;
+    int64_t sq[4], sk[4], sv[4], so[4], sm[4];   // (b, h, l, d); sm = mask (b, h, lq, lk)
+    float scale;          // as given
+    float scale_log2;     // scale * log2(e): scores are kept in the log2 domain
+    int mask_kind;        // sdpa_mask_kind
+    int group;            // Hq / Hkv
+    // split-K (decode path, and the fp32 flash kernel when it splits keys)
+    int splits;           // 1 = write the output directly
+    int64_t keys_per_split;
+    float* part_o;        // [rows][splits][Dv]   rows = B*Hq*Lq, row = (b*Hq + h)*Lq + i
+    float* part_lse;      // [rows][splits]       log2-domain log-sum-exp, -inf = no key
+};
+
+// Launch shapes chosen by a plan function; the dispatcher checks them against
+// device limits before any launch.
+struct LaunchPlan {
+    dim3 grid;
+    dim3 block;
+    size_t smem_bytes;
+    int splits;
+    int64_t keys_per_split;
+    int variant;          // kernel-specific (decode: row groups per KV head)
+    int aux;              // kernel-specific (decode: 8-row n-tiles per CTA)
+};
+
+struct DeviceInfo {
+    int device;
+    int sm_count;
+    int max_smem_optin;   // bytes per block
+    int cc_major, cc_minor;
+};
+
+// ---- fp32 (and generic) flash kernel on CUDA cores: flash_ffma.cu
+bool ffma_supported(int dtype, int64_t Dqk, int64_t Dv);
+LaunchPlan ffma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev, bool split_keys);
+cudaError_t ffma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, cudaStream_t stream);
+
+// ---- fp16/bf16 split-K decode on mma.sync: decode_mma.cu
+bool decode_mma_supported(int dtype, int64_t Dqk, int64_t Dv);
+LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev);
+cudaError_t decode_mma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, cudaStream_t stream);
+
+// ---- log-sum-exp combine of split-K partials + zero fill: combine.cu
+cudaError_t combine_launch(const AttnParams& p, int dtype, cudaStream_t stream);
+cudaError_t zero_fill_launch(const AttnParams& p, int dtype, cudaStream_t stream);
+
+// ---- fp16/bf16 prefill on tcgen05 / TMEM / TMA: prefill_sm100.cu
+bool prefill_tc_supported(int dtype, int64_t Dqk, int64_t Dv, const AttnParams& p);
+LaunchPlan prefill_tc_plan(const AttnParams& p, int dtype, const DeviceInfo& dev);
+cudaError_t prefill_tc_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, cudaStream_t stream);
+
+// Device error flags of each unit (read and clear; synchronous on `stream`).
+int take_device_error_prefill_tc(cudaStream_t stream);
+
+}  // namespace sdpa

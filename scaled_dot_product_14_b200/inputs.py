@@ -31,11 +31,13 @@ MASK_NONE, MASK_ADDITIVE, MASK_BOOL, MASK_CAUSAL = 0, 1, 2, 3
 # ----------------------------------------------------------------------------- dtype storage
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float32 to bfloat16 (nearest, ties to even); returns uint16 bits."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    is_nan = np.isnan(np.asarray(x, dtype=np.float32))
-    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    r = r.astype(np.uint16)
-    r[is_nan] = 0x7FC0
+    f = np.ascontiguousarray(x, dtype=np.float32)
+    u = f.view(np.uint32)
+    # finite and infinite values stay below 2^32 after the rounding increment
+    r = ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)
+    nan = np.isnan(f)
+    if nan.any():
+        r[nan] = 0x7FC0
     return r
 
 
@@ -125,7 +127,8 @@ def make_case(seed: int, B: int, Hq: int, Hkv: int, Lq: int, Lk: int, Dqk: int, 
               dtype: int = BF16, mask: str = "none", layout: str = "bhld", p_keep: float = 0.9,
               scale: float | None = None) -> Case:
     """Seeded N(0,1) case.  mask in {"none", "causal", "decode_additive",
-    "additive" ([B,1,Lq,Lk] U(-1,0)), "additive_full" ([B,Hq,Lq,Lk]), "bool" ([1,1,Lq,Lk]),
+    "additive" ([B,1,Lq,Lk] U(-1,0)), "additive_bcast" ([1,1,Lq,Lk]), "additive_full" ([B,Hq,Lq,Lk]),
+    "bool" ([1,1,Lq,Lk]),
     "bool_full" ([B,Hq,Lq,Lk])}."""
     Dv = Dqk if Dv is None else Dv
     rng = np.random.default_rng(seed)
@@ -150,6 +153,9 @@ def make_case(seed: int, B: int, Hq: int, Hkv: int, Lq: int, Lk: int, Dqk: int, 
     elif mask == "additive":
         m = rng.uniform(-1.0, 0.0, size=(B, 1, Lq, Lk)).astype(np.float32)
         mk, mbuf, mst = MASK_ADDITIVE, to_storage(m.reshape(-1), dtype), (Lq * Lk, 0, Lk, 1)
+    elif mask == "additive_bcast":
+        m = rng.uniform(-1.0, 0.0, size=(Lq, Lk)).astype(np.float32)
+        mk, mbuf, mst = MASK_ADDITIVE, to_storage(m.reshape(-1), dtype), (0, 0, Lk, 1)
     elif mask == "additive_full":
         m = rng.uniform(-1.0, 0.0, size=(B, Hq, Lq, Lk)).astype(np.float32)
         mk, mbuf, mst = MASK_ADDITIVE, to_storage(m.reshape(-1), dtype), (Hq * Lq * Lk, Lq * Lk, Lk, 1)

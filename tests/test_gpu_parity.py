@@ -1,0 +1,296 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle, on
+the same seeded stored inputs, element by element (every row at sizes the
+oracle finishes in seconds; seeded sampled rows at full sizes).
+
+Workloads follow the pages: the MLX issue #3585 linspace case, the decode
+shapes of MLX issue #3885 (d=256 32q/8kv and d=512 32q/4kv, additive mask, qL=1,
+seqK 1k/4k; d=512 prefill), the head-dim-72 prefill of MLX PR #4330 (B=1, 16
+heads, N=8192), and that PR's coverage sweep (dtypes x masks, aligned and
+unaligned lengths)."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import scaled_dot_product_14_b200 as S
+from scaled_dot_product_14_b200 import inputs as I
+
+from gpu_util import GpuCase, compare, oracle_rows, run_and_check, TOL
+
+pytestmark = pytest.mark.gpu
+
+DIMS = [(64, 64), (72, 72), (80, 80), (96, 96), (128, 128), (192, 128), (256, 256), (512, 512)]
+DTYPES = [I.F32, I.F16, I.BF16]
+MASKS = ["none", "additive", "bool", "causal"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from scaled_dot_product_14_b200 import build
+    import oracle
+    build.build()
+    oracle.build()
+    assert torch.cuda.is_available()
+    cap = torch.cuda.get_device_capability()
+    assert cap == (10, 0), f"expected a B200 (sm_100), got {cap}"
+
+
+def path_of(c):
+    st, path = S.sdpa_supported(c.B, c.Hq, c.Hkv, c.Lq, c.Lk, c.Dqk, c.Dv, c.all_strides16, c.mask_kind,
+                                c.mask_strides if c.mask is not None else None, c.dtype)
+    assert st == 0
+    return path
+
+
+# ---------------------------------------------------------------- MLX issue #3585 linspace case
+def _page1_case(layout_view: str, values: np.ndarray):
+    """values: float32 [B, L, H, D]."""
+    B, L, H, D = values.shape
+    if layout_view == "blhd_strided":        # the [B,L,H,D] buffer passed with its own strides
+        buf, st = values.reshape(-1), I.strides_for("blhd", B, H, L, D)
+        ost = I.strides_for("blhd", B, H, L, D)
+    else:                                    # a contiguous [B,H,L,D] copy
+        buf = np.ascontiguousarray(values.transpose(0, 2, 1, 3)).reshape(-1)
+        st = ost = I.strides_for("bhld", B, H, L, D)
+    return I.Case(B, H, H, L, L, D, D, I.F32, buf, buf.copy(), buf.copy(), st * 3, ost, I.default_scale(D),
+                  layout="blhd" if layout_view == "blhd_strided" else "bhld")
+
+
+@pytest.mark.parametrize("view", ["blhd_strided", "bhld_copy"])
+def test_page1_linspace(view):
+    x = I.page1_linspace((2, 82, 8, 64))
+    c = _page1_case(view, x)
+    (mx, mean), got = run_and_check(c, label=f"page1 {view}")
+    assert path_of(c) == S.SDPA_PATH_PREFILL
+
+
+def test_page1_normal_copy():
+    x = np.random.default_rng(1000).standard_normal((2, 82, 8, 64), dtype=np.float32)
+    run_and_check(_page1_case("blhd_strided", x), label="page1 N(0,1)")
+
+
+def test_page1_printed_differences_through_gpu():
+    """The GPU reproduces both printed max-differences of MLX issue #3585: fed the
+    buffer with its true [B,L,H,D] strides it gives correct attention (0.3308013
+    from the whole-array-softmax "manual"), and fed the same buffer declared as
+    [B, H=82, L=8, D] it gives the misread-layout output (0.4969254)."""
+    gold = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "mlx3585_linspace.json")))["printed"]
+    x = I.page1_linspace((2, 82, 8, 64))
+    xt = x.astype(np.float64).transpose(0, 2, 1, 3)
+    sc = xt @ xt.transpose(0, 1, 3, 2) * (64 ** -0.5)
+    w = np.exp(sc - sc.max())
+    G = ((w / w.sum()) @ xt).transpose(0, 2, 1, 3)
+    g = GpuCase(_page1_case("blhd_strided", x))
+    assert g.run() == 0
+    C = g.output().transpose(0, 2, 1, 3)
+    assert abs(np.abs(G - C).max() - gold["manual_vs_pytorch_fused_max_diff"]) < 1e-5
+    buf = x.reshape(-1)
+    st = I.strides_for("bhld", 2, 82, 8, 64)
+    mis = I.Case(2, 82, 82, 8, 8, 64, 64, I.F32, buf, buf, buf, st * 3, st, I.default_scale(64))
+    gm = GpuCase(mis)
+    assert gm.run() == 0
+    M = gm.output()
+    assert abs(np.abs(G - M).max() - gold["manual_vs_fused_max_diff"]) < 1e-5
+
+
+# ---------------------------------------------------------------- decode workloads (MLX issue #3885)
+@pytest.mark.parametrize("kL", [1024, 4096])
+def test_decode_d256_gqa4_additive(kL):
+    c = I.make_case(1001, 1, 32, 8, 1, kL, 256, dtype=I.BF16, mask="decode_additive")
+    assert path_of(c) == S.SDPA_PATH_DECODE
+    before = S.sdpa_get_counters()
+    run_and_check(c, label=f"decode d256 kL={kL}")
+    after = S.sdpa_get_counters()
+    assert after["decode_mma_launches"] == before["decode_mma_launches"] + 1
+
+
+@pytest.mark.parametrize("kL", [1024, 4096])
+@pytest.mark.parametrize("mask", ["none", "decode_additive"])
+def test_decode_d512_gqa8(kL, mask):
+    c = I.make_case(1002, 1, 32, 4, 1, kL, 512, dtype=I.BF16, mask=mask)
+    run_and_check(c, label=f"decode d512 kL={kL} {mask}")
+
+
+def test_prefill_d512_causal_4096():
+    c = I.make_case(1002, 1, 32, 4, 4096, 4096, 512, dtype=I.BF16, mask="causal")
+    rows = I.sample_rows(1002, 1, 32, 4096, 96)
+    run_and_check(c, rows=rows, label="prefill d512 causal L=4096")
+
+
+# ---------------------------------------------------------------- head dim 72 prefill (MLX PR #4330)
+@pytest.mark.parametrize("dtype,mask", [(I.BF16, "none"), (I.F16, "none"), (I.BF16, "bool")])
+def test_prefill_d72_8192(dtype, mask):
+    c = I.make_case(1003, 1, 16, 16, 8192, 8192, 72, dtype=dtype, mask=mask, layout="blhd", p_keep=0.9)
+    rows = I.sample_rows(1003, 1, 16, 8192, 64)
+    run_and_check(c, rows=rows, label=f"prefill d72 {dtype} {mask}")
+
+
+# ---------------------------------------------------------------- the coverage sweep
+def _sweep_case(D, Dv, dtype, mask, L, seed, B=2):
+    # at the largest size the additive mask is broadcast over the batch ([1,1,L,L]) to bound host memory
+    m = {"additive": "additive" if L < 16384 else "additive_bcast", "bool": "bool", "causal": "causal",
+         "none": "none"}[mask]
+    return I.make_case(seed, B, 32, 8, L, L, D, Dv, dtype=dtype, mask=m)
+
+
+@pytest.mark.parametrize("D,Dv", DIMS)
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("mask", MASKS)
+def test_sweep_L128_full(D, Dv, dtype, mask):
+    c = _sweep_case(D, Dv, dtype, mask, 128, 1004)
+    run_and_check(c, label=f"sweep L=128 D={D} dt={dtype} {mask}")
+
+
+@pytest.mark.parametrize("D,Dv", DIMS)
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("mask", MASKS)
+def test_sweep_L2048_sampled(D, Dv, dtype, mask):
+    c = _sweep_case(D, Dv, dtype, mask, 2048, 1005)
+    rows = I.sample_rows(1005, 2, 32, 2048, 48)
+    run_and_check(c, rows=rows, label=f"sweep L=2048 D={D} dt={dtype} {mask}")
+
+
+@pytest.mark.parametrize("D,Dv", DIMS)
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_sweep_L16384_sampled(D, Dv, dtype):
+    # one mask per (dim, dtype), cycling, to bound the run time of the largest size
+    mask = MASKS[(DIMS.index((D, Dv)) + DTYPES.index(dtype)) % 4]
+    c = _sweep_case(D, Dv, dtype, mask, 16384, 1006, B=1)
+    rows = I.sample_rows(1006, 1, 32, 16384, 24)
+    run_and_check(c, rows=rows, label=f"sweep L=16384 D={D} dt={dtype} {mask}")
+
+
+@pytest.mark.parametrize("D,Dv", DIMS)
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("mask", MASKS)
+def test_chunked_query_consistency(D, Dv, dtype, mask):
+    """mlxcel issue #1065, "The four failing tests": qL=4 in chunks of 1 must equal
+    the unchunked call; each chunk is a decode call on a key prefix (causal,
+    bottom-right) and every result is checked against the oracle."""
+    lq, lk = 4, 300
+    c = I.make_case(1007, 2, 32, 8, lq, lk, D, Dv, dtype=dtype,
+                    mask={"additive": "additive", "bool": "bool_full"}.get(mask, mask))
+    (_, _), full = run_and_check(c, label="unchunked")
+    tmax, _ = TOL[dtype]
+    for a in range(lq):
+        import dataclasses
+        kv = lk - lq + a + 1 if mask == "causal" else lk
+        st = c.strides
+        sub = dataclasses.replace(
+            c, Lq=1, Lk=kv, q=c.q[a * st[2]:], mask_kind=c.mask_kind,
+            mask=None if c.mask is None else c.mask[a * c.mask_strides[2]:])
+        (_, _), part = run_and_check(sub, label=f"chunk {a}")
+        assert np.abs(part[:, :, 0] - full[:, :, a]).max() <= 2 * tmax
+
+
+# ---------------------------------------------------------------- edge cases
+@pytest.mark.parametrize("Lq", [1, 2, 7, 8, 9, 16, 17, 127, 129])
+@pytest.mark.parametrize("Lk", [1, 7, 127, 129])
+@pytest.mark.parametrize("dtype,D,mask", [(I.BF16, 128, "causal"), (I.F16, 72, "none"), (I.F32, 96, "bool_full"),
+                                          (I.BF16, 512, "additive")])
+def test_ragged_lengths(Lq, Lk, dtype, D, mask):
+    c = I.make_case(1100 + Lq * 7 + Lk, 2, 4, 2, Lq, Lk, D, dtype=dtype, mask=mask, p_keep=0.7)
+    run_and_check(c, label=f"Lq={Lq} Lk={Lk}")
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16, 32])
+@pytest.mark.parametrize("Lq", [1, 8, 40])
+def test_gqa_ratios(G, Lq):
+    c = I.make_case(1200 + G, 2, 2 * G, 2, Lq, 333, 128, dtype=I.BF16, mask="causal" if Lq > 1 else "none")
+    run_and_check(c, label=f"G={G} Lq={Lq}")
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_many_decode_rows(dtype):
+    # 64 query heads on one KV head, 8 queries: 512 rows per group -> several row groups per CTA grid
+    c = I.make_case(1300, 2, 64, 1, 8, 1000, 128, dtype=dtype, mask="causal")
+    run_and_check(c, label="MQA qL=8")
+
+
+@pytest.mark.parametrize("Lq", [1, 33])
+def test_no_keys_gives_zeros(Lq):
+    c = I.make_case(1400, 1, 4, 2, Lq, 0, 64, dtype=I.BF16)
+    g = GpuCase(c)
+    assert g.run() == 0
+    assert np.all(g.output() == 0.0)
+
+
+def test_empty_batch_launches_nothing():
+    c = I.make_case(1401, 0, 4, 2, 16, 16, 64, dtype=I.BF16)
+    before = S.sdpa_get_counters()
+    g = GpuCase(c)
+    assert g.run() == 0
+    after = S.sdpa_get_counters()
+    assert after["empty_calls"] == before["empty_calls"] + 1
+    assert S.sdpa_last_launch_count() == 0
+
+
+@pytest.mark.parametrize("Lq", [8, 40])
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_causal_more_queries_than_keys(Lq, dtype):
+    """Bottom-right alignment: queries i < Lq - Lk see no key and output zeros."""
+    c = I.make_case(1402, 1, 4, 2, Lq, 5, 64, dtype=dtype, mask="causal")
+    (_, _), got = run_and_check(c, label="causal Lq>Lk")
+    assert np.all(got[:, :, :Lq - 5] == 0.0)
+
+
+@pytest.mark.parametrize("Lq", [1, 24])
+def test_fully_masked_rows_are_zero(Lq):
+    c = I.make_case(1403, 1, 4, 2, Lq, 100, 256, dtype=I.BF16, mask="bool")
+    c.mask.reshape(Lq, 100)[0, :] = 0
+    (_, _), got = run_and_check(c, label="masked row")
+    assert np.all(got[:, :, 0] == 0.0)
+    c2 = I.make_case(1404, 1, 4, 2, Lq, 100, 64, dtype=I.F16, mask="additive")
+    m = I.storage_to_f32(c2.mask, c2.dtype).reshape(1, 1, Lq, 100)
+    m[0, 0, 0, :] = -np.inf
+    c2.mask = I.to_storage(m.reshape(-1), c2.dtype)
+    (_, _), got2 = run_and_check(c2, label="-inf row")
+    assert np.all(got2[:, :, 0] == 0.0)
+
+
+@pytest.mark.parametrize("Lq", [1, 100])
+def test_strided_views(Lq):
+    """q as a head-slice of a wider tensor, out into a strided sub-view."""
+    B, Hq, Hkv, Lk, D = 2, 8, 4, 150, 128
+    big = I.make_case(1500, B, 2 * Hq, Hkv, Lq, Lk, D, dtype=I.BF16, layout="blhd")
+    import dataclasses
+    st = list(big.strides)
+    # take every other query head: head stride doubles, count halves
+    st[1] = 2 * st[1]
+    ost = (Lq * Hq * 2 * D, 2 * D, Hq * 2 * D, 1)   # out: [B, L, 2*Hq, D] buffer, every other head
+    c = dataclasses.replace(big, Hq=Hq, strides=tuple(st), out_strides=ost)
+    run_and_check(c, label="strided view")
+
+
+def test_layouts_agree_on_gpu():
+    a = I.make_case(1600, 2, 8, 2, 200, 200, 96, dtype=I.BF16, layout="bhld", mask="causal")
+    b = I.make_case(1600, 2, 8, 2, 200, 200, 96, dtype=I.BF16, layout="blhd", mask="causal")
+    (_, _), ga = run_and_check(a, label="bhld")
+    (_, _), gb = run_and_check(b, label="blhd")
+    assert np.abs(ga - gb).max() <= 1e-6
+
+
+def test_fp32_keeps_fp32_precision():
+    """mlxcel issue #1065: fp32 error near 2^-10 = 9.77e-4 would mean reduced
+    internal precision; the fp32 path must stay far below it on both paths."""
+    for Lq in (1, 64):
+        c = I.make_case(1700 + Lq, 1, 8, 2, Lq, 4096, 128, dtype=I.F32, mask="causal")
+        (mx, mean), _ = run_and_check(c, label=f"fp32 Lq={Lq}")
+        assert mx < 1e-5 < 2.0 ** -10
+
+
+def test_repeat_calls_are_deterministic():
+    c = I.make_case(1800, 1, 32, 8, 1, 4096, 256, dtype=I.BF16, mask="decode_additive")
+    g = GpuCase(c)
+    assert g.run() == 0
+    a = g.output().copy()
+    assert g.run() == 0
+    b = g.output()
+    assert np.array_equal(a, b)
+
+
+def test_counters_invariant():
+    c = S.sdpa_get_counters()
+    assert c["calls"] == c["prefill_calls"] + c["decode_calls"] + c["empty_calls"] + c["rejected_calls"]

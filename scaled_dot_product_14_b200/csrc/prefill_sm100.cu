@@ -1,17 +1,573 @@
-// prefill_sm100.cu -- fp16/bf16 prefill on tcgen05 tensor cores (placeholder
-// until the TMA + TMEM kernel lands: reports no coverage).
+// prefill_sm100.cu -- fp16/bf16 prefill attention on 5th-generation tensor
+// cores: TMA tile loads, tcgen05.mma with TMEM accumulators, fused online
+// softmax (fp32) with masks, causal tile skipping.
+//
+// The "full" (qL > 8) path of MLX issue #3885 ("Metal SDPA: no fused path for
+// head_dim=512 ..."), section "Current routing", for every head dim of that
+// section plus 72 (MLX PR #4330, "Support head dimension 72 in Metal full
+// attention").  The pages' kernels tile the head dim on 8x8 simdgroup
+// fragments (Steel, TD=9 at d=72) or kU=16 (NAX, which needs d % 32 == 0).
+// Here the MMA K step is 16, so d=72 is padded to 80 inside the MMA only: the
+// TMA descriptors keep the true extent and the hardware zero-fills columns
+// 72..79, costing no memory traffic (that PR's section "Benchmarks" shows why
+// head dim 72 must not fall back to the unfused path).
+//
+// One CTA computes a 128-row query tile of one (batch, query head):
+//   warp 0      TMA producer: Q once, then K and V as 16 KB chunks (128 keys
+//               x 64 head-dim elements, 128-byte swizzle) into one ring, in
+//               the order the MMAs consume them;
+//   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of two TMEM
+//               S buffers (double-buffered), then O += P V with P read from
+//               TMEM (it overwrites its own S buffer) and O kept in TMEM;
+//   warps 2..5  softmax: thread t owns query row t (its TMEM lane), scales,
+//               masks, keeps the running max / sum in fp32 (log2 domain),
+//               writes P as 16-bit pairs back to TMEM, rescales O in TMEM
+//               only when its row maximum grew by more than 2^8 (the result
+//               is exact either way after the final 1/l), and finally
+//               normalises O and stores it through the output strides.
+// Head dim 512 (MLX issue #3885, section "Requests": a split-D variant):
+// O for 128 rows x 512 fp32 columns would fill all of TMEM, so two CTAs share
+// a query tile and each produces 256 of the value columns (S is computed by
+// both; the tensor work is 1.5x the algorithmic count for that head dim).
+// Every mbarrier wait is bounded (globaltimer); on expiry the kernel records
+// an error code, drains its TMA loads and MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
 
 namespace sdpa {
+namespace {
 
-bool prefill_tc_supported(int, int64_t, int64_t, const AttnParams&) { return false; }
-LaunchPlan prefill_tc_plan(const AttnParams&, int, const DeviceInfo&) { return LaunchPlan{}; }
-cudaError_t prefill_tc_launch(const AttnParams&, int, const LaunchPlan&, cudaStream_t) {
-    return cudaErrorNotSupported;
+constexpr int kBM = 128;               // query rows per CTA (UMMA M)
+constexpr int kBN = 128;               // keys per tile (UMMA N of S)
+constexpr int kChunk = kBN * 128;      // one ring slot: 128 rows x 64 head-dim elements (128-byte swizzle)
+constexpr int kThreads = 192;          // 6 warps
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
+
+__host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// DQK: q/k head dim; DVC: value columns this CTA produces (Dv, or Dv/2 when the
+// pair of CTAs splits Dv: head dim 512); NSLOT: ring slots; SPLIT: CTAs per query tile.
+template <int DQK, int DVC, int NSLOT, int SPLIT>
+struct TcCfg {
+    static constexpr int NBQ = cdiv(DQK, 64);        // Q / K chunks
+    static constexpr int NBV = cdiv(DVC, 64);        // V chunks per CTA
+    static constexpr int KSTEPS = cdiv(DQK, 16);     // K steps of S = Q K^T
+    static constexpr int DVP = cdiv(DVC, 16) * 16;   // O columns in TMEM
+    static constexpr int Q_BYTES = NBQ * kBM * 128;
+    static constexpr int OFF_RING = Q_BYTES;
+    static constexpr int OFF_BAR = OFF_RING + NSLOT * kChunk;
+    static constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 + 2 + 1 + 1;
+    static constexpr int SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 1024;   // + TMEM slot + alignment slack
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr int O_COL = 2 * kBN;
+    static_assert(O_COL + DVP <= 512, "TMEM budget: two S buffers and O");
+    static_assert(NSLOT >= 2, "ring depth");
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+// Which tensor-map dimension carries the sequence, head and batch index
+// (the host orders the three by stride); pos 0 means "always coordinate 0".
+struct MapAxes {
+    int l_pos, h_pos, b_pos;
+};
+
+struct TcParams {
+    AttnParams p;
+    MapAxes q_ax, k_ax, v_ax;
+    int q_tiles;
+};
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
 }
+
+// Bounded wait on an mbarrier phase: ~2 s, then the error flag and false.
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int code) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer() - t0 > 2000000000ull) {
+            atomicCAS(&g_sdpa_device_error, 0, code);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, uint64_t* bar, const MapAxes& ax,
+                                         int d0, int l, int h, int b) {
+    int c[4] = {d0, 0, 0, 0};
+    if (ax.l_pos) c[ax.l_pos] = l;
+    if (ax.h_pos) c[ax.h_pos] = h;
+    if (ax.b_pos) c[ax.b_pos] = b;
+    tma_load_4d(dst, map, bar, c[0], c[1], c[2], c[3]);
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&o)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]), "=r"(o[7]), "=r"(o[8]),
+          "=r"(o[9]), "=r"(o[10]), "=r"(o[11]), "=r"(o[12]), "=r"(o[13]), "=r"(o[14]), "=r"(o[15])
+        : "r"(taddr));
+}
+
+template <typename T, int DQK, int DVC, int NSLOT, int SPLIT>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const TcParams tp) {
+    using C = TcCfg<DQK, DVC, NSLOT, SPLIT>;
+    constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    const AttnParams& p = tp.p;
+
+    extern __shared__ unsigned char smem_dyn[];
+    unsigned char* smem =
+        reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t ring = s_base + C::OFF_RING;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* bar_q = bars;
+    uint64_t* bar_full = bars + 1;              // [NSLOT]
+    uint64_t* bar_empty = bar_full + NSLOT;     // [NSLOT]
+    uint64_t* bar_s_full = bar_empty + NSLOT;   // [2]
+    uint64_t* bar_p_full = bar_s_full + 2;      // [2]
+    uint64_t* bar_o_done = bar_p_full + 2;
+    uint64_t* bar_drain = bar_o_done + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // causal work is heaviest for the last query tiles: run them first
+    const int tile_idx = (int)blockIdx.x / SPLIT;
+    const int half = (int)blockIdx.x % SPLIT;
+    const int qt = (p.mask_kind == 3) ? (tp.q_tiles - 1 - tile_idx) : tile_idx;
+    const int hq = blockIdx.y, b = blockIdx.z;
+    const int hkv = hq / p.group;
+    const int64_t q0 = (int64_t)qt * kBM;
+    const int dv0 = half * DVC;   // first value column of this CTA
+
+    // number of key tiles this query tile needs (causal: up to the diagonal)
+    int64_t kv_len = p.Lk;
+    if (p.mask_kind == 3) {
+        const int64_t last = q0 + kBM - 1 + p.Lk - p.Lq;   // last key that row q0+127 sees
+        kv_len = last < 0 ? 0 : (last + 1 < p.Lk ? last + 1 : p.Lk);
+    }
+    const int n_tiles = (int)((kv_len + kBN - 1) / kBN);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < NSLOT; ++s) {
+            mbar_init(bar_full + s, 1);
+            mbar_init(bar_empty + s, 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar_s_full + s, 1);
+            mbar_init(bar_p_full + s, 128);
+        }
+        mbar_init(bar_o_done, 1);
+        mbar_init(bar_drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        // Chunks go through the ring in exactly the order the MMA warp consumes
+        // them: K(0), then per tile j: K(j+1), V(j).
+        if (lane == 0 && n_tiles > 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
+            for (int c = 0; c < C::NBQ; ++c) tma_load(s_base + c * kChunk, &tmQ, bar_q, tp.q_ax, c * 64, (int)q0, hq, b);
+            int seq = 0;
+            bool ok = true;
+            auto put = [&](const CUtensorMap* map, const MapAxes& ax, int d0, int j) -> bool {
+                const int slot = seq % NSLOT;
+                if (!wait_phase(bar_empty + slot, ((seq / NSLOT) & 1) ^ 1, kErrWaitSlot)) return false;
+                mbar_arrive_expect_tx(bar_full + slot, kChunk);
+                tma_load(ring + slot * kChunk, map, bar_full + slot, ax, d0, j * kBN, hkv, b);
+                ++seq;
+                return true;
+            };
+            for (int c = 0; c < C::NBQ && ok; ++c) ok = put(&tmK, tp.k_ax, c * 64, 0);
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                if (j + 1 < n_tiles)
+                    for (int c = 0; c < C::NBQ && ok; ++c) ok = put(&tmK, tp.k_ax, c * 64, j + 1);
+                for (int c = 0; c < C::NBV && ok; ++c) ok = put(&tmV, tp.v_ax, dv0 + c * 64, j);
+            }
+            if (!ok) {
+                // drain: every issued load must land before the CTA's shared memory goes away
+                wait_phase(bar_q, 0, kErrWaitTmaLoad);
+                for (int x = (seq > NSLOT ? seq - NSLOT : 0); x < seq; ++x)
+                    wait_phase(bar_full + x % NSLOT, (x / NSLOT) & 1, kErrWaitTmaLoad);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && n_tiles > 0) {
+            constexpr uint32_t idS = umma_idesc_f16(kBF16 ? 1 : 0, kBM, kBN, 0, 0);
+            int seq = 0;
+            bool ok = wait_phase(bar_q, 0, kErrWaitTmaLoad);
+            tc_fence_after();
+            auto issue_s = [&](int j) -> bool {   // S_j = Q K_j^T into TMEM buffer j & 1
+                const uint32_t d = tmem + (uint32_t)((j & 1) * kBN);
+#pragma unroll
+                for (int c = 0; c < C::NBQ; ++c) {
+                    const int slot = seq % NSLOT;
+                    if (!wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        if (c * 4 + k4 >= C::KSTEPS) break;
+                        const uint64_t da = umma_desc_sw128(s_base + c * kChunk + k4 * 32, 16, 1024);
+                        const uint64_t db = umma_desc_sw128(ring + slot * kChunk + k4 * 32, 16, 1024);
+                        umma_ss(d, da, db, idS, (c > 0 || k4 > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar_empty + slot);
+                    ++seq;
+                }
+                umma_commit(bar_s_full + (j & 1));
+                return true;
+            };
+            auto issue_pv = [&](int j) -> bool {   // O += P_j V_j, P_j read from TMEM
+                const uint32_t a_tmem = tmem + (uint32_t)((j & 1) * kBN);
+#pragma unroll
+                for (int c = 0; c < C::NBV; ++c) {
+                    const int slot = seq % NSLOT;
+                    if (!wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
+                    tc_fence_after();
+                    constexpr int kLastN = C::DVP - 64 * (C::NBV - 1);
+                    const uint32_t idPV =
+                        umma_idesc_f16(kBF16 ? 1 : 0, kBM, (c == C::NBV - 1) ? kLastN : 64, 0, 1);
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk) {
+                        const uint64_t db = umma_desc_sw128(ring + slot * kChunk + kk * 2048, kChunk, 1024);
+                        umma_ts(tmem + C::O_COL + c * 64, a_tmem + kk * 8, db, idPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar_empty + slot);
+                    ++seq;
+                }
+                umma_commit(bar_o_done);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                if (j + 1 < n_tiles) {
+                    // S_{j+1} reuses the TMEM buffer P_{j-1} was read from: wait for PV_{j-1}
+                    if (j >= 1 && !(ok = wait_phase(bar_o_done, (j - 1) & 1, kErrWaitMma))) break;
+                    if (!(ok = issue_s(j + 1))) break;
+                }
+                if (!(ok = wait_phase(bar_p_full + (j & 1), (j >> 1) & 1, kErrWaitSoftmax))) break;
+                tc_fence_after();
+                if (!(ok = issue_pv(j))) break;
+            }
+            // every MMA issued by this thread completes before TMEM can be freed
+            umma_commit(bar_drain);
+            wait_phase(bar_drain, 0, kErrWaitMma);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax / correction / epilogue
+        const int quad = warp & 3;   // warps 2,3,4,5 -> TMEM lane quadrants 2,3,0,1
+        const int r = quad * 32 + lane;
+        const int64_t i = q0 + r;
+        const bool row_ok = i < p.Lq;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const int64_t causal_lim = i + p.Lk - p.Lq;
+        const float log2e = 1.4426950408889634f;
+        const T* mask_t = reinterpret_cast<const T*>(p.mask);
+        const uint8_t* mask_b = reinterpret_cast<const uint8_t*>(p.mask);
+        const int64_t mrow = (int64_t)b * p.sm[0] + (int64_t)hq * p.sm[1] + i * p.sm[2];
+
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            const int buf = j & 1;
+            ok = __all_sync(0xffffffffu, wait_phase(bar_s_full + buf, (j >> 1) & 1, kErrWaitMma));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sr[kBN];
+#pragma unroll
+            for (int c = 0; c < kBN / 32; ++c)
+                tmem_ld32(tmem + lane_off + buf * kBN + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
+            tmem_wait_ld();
+
+            const int64_t kbase = (int64_t)j * kBN;
+            float mloc = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kBN; ++c) {
+                const int64_t key = kbase + c;
+                float x = __uint_as_float(sr[c]) * p.scale_log2;
+                bool keep = row_ok && key < p.Lk;
+                if (p.mask_kind == 3) {
+                    keep = keep && key <= causal_lim;
+                } else if (p.mask_kind == 1) {
+                    if (keep) x += Elem<T>::to_float(mask_t[mrow + key * p.sm[3]]) * log2e;
+                } else if (p.mask_kind == 2) {
+                    keep = keep && mask_b[mrow + key * p.sm[3]] != 0;
+                }
+                x = keep ? x : -INFINITY;
+                sr[c] = __float_as_uint(x);
+                mloc = fmaxf(mloc, x);
+            }
+            const float m_new = fmaxf(m_ref, mloc);
+            float alpha = 1.f;
+            bool rescale = false;
+            if (m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + kRescaleThreshold)) {
+                rescale = (m_ref != -INFINITY);   // before the first finite max, O holds zeros
+                alpha = rescale ? fast_exp2(m_ref - m_new) : 0.f;
+                m_ref = m_new;
+            }
+            const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+            l *= alpha;
+            uint32_t pr[kBN / 2];
+#pragma unroll
+            for (int c = 0; c < kBN / 2; ++c) {
+                const float p0 = fast_exp2(__uint_as_float(sr[2 * c]) - m_use);
+                const float p1 = fast_exp2(__uint_as_float(sr[2 * c + 1]) - m_use);
+                l += p0 + p1;
+                pr[c] = pack2<T>(p0, p1);
+            }
+#pragma unroll
+            for (int c = 0; c < kBN / 64; ++c)
+                tmem_st32(tmem + lane_off + buf * kBN + c * 32, *reinterpret_cast<uint32_t(*)[32]>(pr + c * 32));
+            tmem_wait_st();
+
+            if (j > 0) {
+                ok = __all_sync(0xffffffffu, wait_phase(bar_o_done, (j - 1) & 1, kErrWaitMma));
+                if (!ok) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, rescale)) {
+                    const float f = rescale ? alpha : 1.f;
+#pragma unroll
+                    for (int c = 0; c < C::DVP / 16; ++c) {
+                        uint32_t o[16];
+                        tmem_ld16(tmem + lane_off + C::O_COL + c * 16, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * f);
+                        tmem_st16(tmem + lane_off + C::O_COL + c * 16, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar_p_full + buf);
+        }
+
+        // epilogue: O / l -> dtype, stored through the output strides
+        if (ok && n_tiles > 0)
+            ok = __all_sync(0xffffffffu, wait_phase(bar_o_done, (n_tiles - 1) & 1, kErrWaitMma));
+        tc_fence_after();
+        T* og = reinterpret_cast<T*>(p.out) + (int64_t)b * p.so[0] + (int64_t)hq * p.so[1] + i * p.so[2] + dv0;
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+        for (int c = 0; c < C::DVP / 16; ++c) {
+            uint32_t o[16];
+            if (n_tiles > 0 && ok) {
+                tmem_ld16(tmem + lane_off + C::O_COL + c * 16, o);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int u = 0; u < 16; ++u) o[u] = 0u;
+            }
+            uint4 w[2];
+            uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                wp[u] = pack2<T>(__uint_as_float(o[2 * u]) * inv, __uint_as_float(o[2 * u + 1]) * inv);
+            if (row_ok) {
+                if (c * 16 < DVC) *reinterpret_cast<uint4*>(og + c * 16) = w[0];
+                if (c * 16 + 8 < DVC) *reinterpret_cast<uint4*>(og + c * 16 + 8) = w[1];
+            }
+        }
+    }
+
+    // teardown: every role has drained its asynchronous work
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// A 4-D tiled map (d, then the sequence / head / batch axes in increasing
+// stride order; an axis of extent 1 or stride 0 is pinned to coordinate 0),
+// 128-byte swizzle, box = 64 elements x box_rows rows, zero fill out of bounds.
+bool make_map(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L, int64_t H,
+              int64_t B, const int64_t* st, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const int64_t esz = 2;
+    struct Axis {
+        int which;   // 0 = l, 1 = h, 2 = b
+        int64_t ext, stride;
+    } axes[3] = {{0, L, st[2] * esz}, {1, H, st[1] * esz}, {2, B, st[0] * esz}};
+    // degenerate axes go last with a stride past every other axis
+    int64_t span = ((D * esz + 15) / 16) * 16;
+    for (auto& a : axes)
+        if (a.ext > 1 && a.stride > 0 && a.stride * a.ext > span) span = a.stride * a.ext;
+    for (auto& a : axes)
+        if (a.ext <= 1 || a.stride == 0) {
+            a.ext = 1;
+            a.stride = ((span + 15) / 16) * 16;
+        }
+    // the sequence axis must stay a real dimension for the box rows; sort by (degenerate, stride)
+    for (int x = 0; x < 3; ++x)
+        for (int y = x + 1; y < 3; ++y) {
+            const bool dx = axes[x].ext == 1 && axes[x].which != 0, dy = axes[y].ext == 1 && axes[y].which != 0;
+            if (dx > dy || (dx == dy && axes[y].stride < axes[x].stride)) {
+                Axis t = axes[x];
+                axes[x] = axes[y];
+                axes[y] = t;
+            }
+        }
+    cuuint64_t gdim[4] = {(cuuint64_t)D, 0, 0, 0};
+    cuuint64_t gstride[3];
+    int pos[3] = {0, 0, 0};
+    for (int x = 0; x < 3; ++x) {
+        gdim[x + 1] = (cuuint64_t)axes[x].ext;
+        gstride[x] = (cuuint64_t)axes[x].stride;
+        pos[axes[x].which] = (axes[x].ext > 1 || axes[x].which == 0) ? x + 1 : 0;
+    }
+    cuuint32_t box[4] = {64, 1, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    for (int x = 0; x < 3; ++x)
+        if (axes[x].which == 0) box[x + 1] = (cuuint32_t)box_rows;
+    const CUtensorMapDataType dt =
+        dtype == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r = fn(map, dt, 4, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    ax->l_pos = pos[0];
+    ax->h_pos = pos[1];
+    ax->b_pos = pos[2];
+    return r == CUDA_SUCCESS;
+}
+
+struct Variant {
+    int split, smem;
+};
+
+template <int DQK, int DVC, int NSLOT, int SPLIT>
+Variant variant_of() {
+    return Variant{SPLIT, TcCfg<DQK, DVC, NSLOT, SPLIT>::SMEM};
+}
+
+// Tile shapes per head dim: (Dqk, Dv per CTA, ring slots, CTAs per query tile).
+#define SDPA_TC_VARIANTS(X)             \
+    X(64, 64, 64, 8, 1)                 \
+    X(72, 72, 72, 8, 1)                 \
+    X(80, 80, 80, 8, 1)                 \
+    X(96, 96, 96, 8, 1)                 \
+    X(128, 128, 128, 8, 1)              \
+    X(192, 128, 128, 10, 1)             \
+    X(256, 256, 256, 10, 1)             \
+    X(512, 512, 256, 6, 2)
+
+Variant pick(int64_t Dqk, int64_t Dv) {
+    switch (Dqk * 1000 + Dv) {
+#define SDPA_TC_PICK(DQ, DVV, DVC, NSL, SP) \
+    case DQ * 1000 + DVV: return variant_of<DQ, DVC, NSL, SP>();
+        SDPA_TC_VARIANTS(SDPA_TC_PICK)
+#undef SDPA_TC_PICK
+        default: return Variant{0, 0};
+    }
+}
+
+template <typename T, int DQK, int DVC, int NSLOT, int SPLIT>
+cudaError_t launch_one(const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const LaunchPlan& plan, cudaStream_t stream) {
+    auto kern = prefill_tc_kernel<T, DQK, DVC, NSLOT, SPLIT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
+    if (e != cudaSuccess) return e;
+    kern<<<plan.grid, plan.block, plan.smem_bytes, stream>>>(mq, mk, mv, tp);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_typed(const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const LaunchPlan& plan, cudaStream_t s) {
+    switch (tp.p.Dqk * 1000 + tp.p.Dv) {
+#define SDPA_TC_LAUNCH(DQ, DVV, DVC, NSL, SP) \
+    case DQ * 1000 + DVV: return launch_one<T, DQ, DVC, NSL, SP>(tp, mq, mk, mv, plan, s);
+        SDPA_TC_VARIANTS(SDPA_TC_LAUNCH)
+#undef SDPA_TC_LAUNCH
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+bool prefill_tc_supported(int dtype, int64_t Dqk, int64_t Dv, const AttnParams& p) {
+    (void)p;
+    if (getenv("SDPA_DISABLE_TCGEN05")) return false;
+    return (dtype == 1 || dtype == 2) && pick(Dqk, Dv).split != 0;
+}
+
+LaunchPlan prefill_tc_plan(const AttnParams& p, int dtype, const DeviceInfo& dev) {
+    (void)dtype;
+    (void)dev;
+    const Variant v = pick(p.Dqk, p.Dv);
+    LaunchPlan plan{};
+    const int64_t q_tiles = (p.Lq + kBM - 1) / kBM;
+    plan.grid = dim3((unsigned)(q_tiles * v.split), (unsigned)p.Hq, (unsigned)p.B);
+    plan.block = dim3(kThreads);
+    // at least 120 KB: one CTA per SM, so a CTA never waits on another CTA's TMEM
+    plan.smem_bytes = (size_t)(v.smem > 120 * 1024 ? v.smem : 120 * 1024);
+    plan.splits = 1;
+    plan.keys_per_split = p.Lk;
+    plan.variant = v.split;
+    plan.aux = (int)q_tiles;
+    return plan;
+}
+
+cudaError_t prefill_tc_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, cudaStream_t stream) {
+    TcParams tp{};
+    tp.p = p;
+    tp.q_tiles = plan.aux;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, &tp.q_ax, p.q, dtype, p.Dqk, p.Lq, p.Hq, p.B, p.sq, kBM) ||
+        !make_map(&mk, &tp.k_ax, p.k, dtype, p.Dqk, p.Lk, p.Hkv, p.B, p.sk, kBN) ||
+        !make_map(&mv, &tp.v_ax, p.v, dtype, p.Dv, p.Lk, p.Hkv, p.B, p.sv, kBN))
+        return cudaErrorInvalidValue;
+    if (dtype == 2) return launch_typed<__nv_bfloat16>(tp, mq, mk, mv, plan, stream);
+    return launch_typed<__half>(tp, mq, mk, mv, plan, stream);
+}
+
 int take_device_error_prefill_tc(cudaStream_t stream) {
     int code = 0;
     if (cudaMemcpyFromSymbolAsync(&code, g_sdpa_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, stream) !=

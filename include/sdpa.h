@@ -123,6 +123,34 @@ int sdpa_forward(const void* q, const void* k, const void* v, void* out,
                  int dtype, void* stream);
 
 /*
+ * sdpa_forward_noalloc -- sdpa_forward for callers that cannot allocate device
+ * memory when they call attention: a process whose memory manager already owns
+ * the whole GPU (a caching allocator, a serving runtime with a fixed memory
+ * budget), or a latency-critical decode loop that must never pay for
+ * cudaMalloc / cudaFree, which can synchronise the device.  The pages describe
+ * no counterpart of this entry point.
+ *
+ * Arguments, layout, validation and result are those of sdpa_forward, but it
+ * covers only the decode path with fp16 / bf16 (Lq <= 8); other problems return
+ * SDPA_ERR_INVALID_ARG (an empty problem returns SDPA_OK).  It allocates
+ * nothing: the split-K partials go to a 4 MiB array compiled into the library,
+ * which every GPU that loads the library holds until the process exits.  A
+ * problem whose partials do not fit (query rows x splits x (Dv + 1) fp32
+ * values, with the split count sdpa_forward would use) returns
+ * SDPA_ERR_TOO_LARGE and launches nothing.  The first call on each device
+ * looks up that array's device address (with the device current); make it
+ * before any stream capture.  All calls on a device share the one array, which
+ * keeps the last call's contents: calls that may overlap on the GPU (different
+ * streams with no ordering between them) race and must not be issued.  The call
+ * counters do not count this entry point.
+ */
+int sdpa_forward_noalloc(const void* q, const void* k, const void* v, void* out,
+                         int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk,
+                         int64_t Dqk, int64_t Dv, const int64_t strides[16], float scale,
+                         int mask_kind, const void* mask, const int64_t mask_strides[4],
+                         int dtype, void* stream);
+
+/*
  * sdpa_supported -- the same validation sdpa_forward runs, without pointers
  * and without launching.  Writes the path that would run (sdpa_path) to
  * *path_out when path_out is not NULL.  Returns an sdpa_status; SDPA_OK means

@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
             L.sdpa_forward.restype = i32
             L.sdpa_forward.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, P64, ctypes.c_float, i32,
                                        vp, P64, i32, vp]
+            L.sdpa_forward_noalloc.restype = i32
+            L.sdpa_forward_noalloc.argtypes = list(L.sdpa_forward.argtypes)
             L.sdpa_supported.restype = i32
             L.sdpa_supported.argtypes = [i64, i64, i64, i64, i64, i64, i64, P64, i32, P64, i32,
                                          ctypes.POINTER(ctypes.c_int)]
@@ -99,6 +101,14 @@ def sdpa_forward(q, k, v, out, B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, scale, mask
     """Calls the C entry point; pointers are ints (device addresses), strides sequences."""
     return lib().sdpa_forward(q, k, v, out, B, Hq, Hkv, Lq, Lk, Dqk, Dv, _i64array(strides, 16),
                               ctypes.c_float(scale), mask_kind, mask, _i64array(mask_strides, 4), dtype, stream)
+
+
+def sdpa_forward_noalloc(q, k, v, out, B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, scale, mask_kind, mask,
+                         mask_strides, dtype, stream) -> int:
+    """The allocation-free decode entry point (same arguments as sdpa_forward)."""
+    return lib().sdpa_forward_noalloc(q, k, v, out, B, Hq, Hkv, Lq, Lk, Dqk, Dv, _i64array(strides, 16),
+                                      ctypes.c_float(scale), mask_kind, mask, _i64array(mask_strides, 4), dtype,
+                                      stream)
 
 
 def sdpa_supported(B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, mask_kind, mask_strides, dtype):

@@ -17,40 +17,59 @@
 namespace sdpa {
 namespace {
 
-constexpr int kRowsPerBlock = 4;   // one warp per query row
+constexpr int kCombineThreads = 128;
+constexpr int kMaxSplitsSmem = 1024;
 
+// One CTA per query row: the split weights go to shared memory once, then
+// each thread accumulates its float4 columns over the splits with independent
+// loads (the loop carries no load-to-load dependency).
 template <typename T>
-__global__ void __launch_bounds__(32 * kRowsPerBlock) combine_kernel(const AttnParams p) {
-    const int lane = threadIdx.x & 31;
-    const int64_t rows = p.B * p.Hq * p.Lq;
-    const int64_t row = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
-    if (row >= rows) return;
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const AttnParams p) {
+    __shared__ float w[kMaxSplitsSmem];
+    __shared__ float red[kCombineThreads / 32];
+    const int64_t row = blockIdx.x;
     const int S = p.splits;
     const float* lse = p.part_lse + row * S;
     float mx = -INFINITY;
-    for (int s = lane; s < S; s += 32) mx = fmaxf(mx, lse[s]);
+    for (int s = threadIdx.x; s < S; s += kCombineThreads) mx = fmaxf(mx, lse[s]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    mx = red[0];
+#pragma unroll
+    for (int wv = 1; wv < kCombineThreads / 32; ++wv) mx = fmaxf(mx, red[wv]);
+    float part = 0.f;
+    for (int s = threadIdx.x; s < S; s += kCombineThreads) {
+        const float ws = (mx == -INFINITY) ? 0.f : exp2f(lse[s] - mx);   // -inf -> 0
+        w[s] = ws;
+        part += ws;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = part;
+    __syncthreads();
+    float wsum = 0.f;
+#pragma unroll
+    for (int wv = 0; wv < kCombineThreads / 32; ++wv) wsum += red[wv];
+    const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
 
     const int64_t i = row % p.Lq, h = (row / p.Lq) % p.Hq, b = row / (p.Lq * p.Hq);
     T* og = reinterpret_cast<T*>(p.out) + b * p.so[0] + h * p.so[1] + i * p.so[2];
     const int nv = (int)(p.Dv / 4);   // float4 chunks (Dv % 4 == 0)
-    for (int c = lane; c < nv; c += 32) {
+    const float4* po = reinterpret_cast<const float4*>(p.part_o + row * S * p.Dv);
+    for (int c = threadIdx.x; c < nv; c += kCombineThreads) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        float wsum = 0.f;
-        if (mx != -INFINITY) {
-            for (int s = 0; s < S; ++s) {
-                const float w = exp2f(lse[s] - mx);   // -inf -> 0
-                if (w == 0.f) continue;
-                const float4 v = *reinterpret_cast<const float4*>(p.part_o + (row * S + s) * p.Dv + c * 4);
-                acc.x += w * v.x;
-                acc.y += w * v.y;
-                acc.z += w * v.z;
-                acc.w += w * v.w;
-                wsum += w;
-            }
+#pragma unroll 8
+        for (int s = 0; s < S; ++s) {
+            const float ws = w[s];
+            const float4 v = po[(int64_t)s * nv + c];
+            acc.x = fmaf(ws, v.x, acc.x);
+            acc.y = fmaf(ws, v.y, acc.y);
+            acc.z = fmaf(ws, v.z, acc.z);
+            acc.w = fmaf(ws, v.w, acc.w);
         }
-        const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
         og[c * 4 + 0] = Elem<T>::from_float(acc.x * inv);
         og[c * 4 + 1] = Elem<T>::from_float(acc.y * inv);
         og[c * 4 + 2] = Elem<T>::from_float(acc.z * inv);
@@ -73,8 +92,9 @@ __global__ void zero_fill_kernel(const AttnParams p) {
 
 cudaError_t combine_launch(const AttnParams& p, int dtype, cudaStream_t stream) {
     const int64_t rows = p.B * p.Hq * p.Lq;
-    const dim3 grid((unsigned)((rows + kRowsPerBlock - 1) / kRowsPerBlock));
-    const dim3 block(32 * kRowsPerBlock);
+    if (p.splits > kMaxSplitsSmem || rows > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)rows);
+    const dim3 block(kCombineThreads);
     switch (dtype) {
         case 0: combine_kernel<float><<<grid, block, 0, stream>>>(p); break;
         case 1: combine_kernel<__half><<<grid, block, 0, stream>>>(p); break;

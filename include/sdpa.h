@@ -133,11 +133,13 @@ int sdpa_forward(const void* q, const void* k, const void* v, void* out,
  * Arguments, layout, validation and result are those of sdpa_forward, but it
  * covers only the decode path with fp16 / bf16 (Lq <= 8); other problems return
  * SDPA_ERR_INVALID_ARG (an empty problem returns SDPA_OK).  It allocates
- * nothing: the split-K partials go to a 4 MiB array compiled into the library,
- * which every GPU that loads the library holds until the process exits.  A
- * problem whose partials do not fit (query rows x splits x (Dv + 1) fp32
- * values, with the split count sdpa_forward would use) returns
- * SDPA_ERR_TOO_LARGE and launches nothing.  The first call on each device
+ * nothing: the split-K partials and the per-group completion counters go to
+ * a 4 MiB array compiled into the library (the counters take its first 64 KiB
+ * and are cleared by each call with a memset on `stream`), which every GPU
+ * that loads the library holds until the process exits.  A problem whose
+ * partials do not fit (query rows x splits x (Dv + 1) fp32 values, with the
+ * split count sdpa_forward would use) returns SDPA_ERR_TOO_LARGE and launches
+ * nothing.  The first call on each device
  * looks up that array's device address (with the device current); make it
  * before any stream capture.  All calls on a device share the one array, which
  * keeps the last call's contents: calls that may overlap on the GPU (different

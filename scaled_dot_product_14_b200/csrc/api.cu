@@ -129,13 +129,18 @@ int device_info(DeviceInfo* out) {
 }
 
 // ---------------------------------------------------------------- split-K workspace
+// Per (device, stream): split-K partials (contents do not outlive a call) and
+// the decode kernel's per-group counters (zero between calls: zeroed when
+// allocated, and every call leaves them zero).
 struct Workspace {
     void* ptr = nullptr;
     size_t bytes = 0;
+    int* counters = nullptr;
+    size_t n_counters = 0;
 };
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
-int workspace(int dev, cudaStream_t stream, size_t bytes, void** out) {
+int workspace(int dev, cudaStream_t stream, size_t bytes, size_t n_counters, void** out, int** counters) {
     std::lock_guard<std::mutex> lk(g_mu);
     Workspace& w = g_ws[{dev, stream}];
     if (w.bytes < bytes) {
@@ -152,7 +157,23 @@ int workspace(int dev, cudaStream_t stream, size_t bytes, void** out) {
         }
         w.bytes = want;
     }
+    if (w.n_counters < n_counters) {
+        if (w.counters) cudaFreeAsync(w.counters, stream);
+        w.counters = nullptr;
+        w.n_counters = 0;
+        const size_t want = n_counters + 1024;
+        cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&w.counters), want * sizeof(int), stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(w.counters, 0, want * sizeof(int), stream);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            w.counters = nullptr;
+            t_last_cuda_error = cudaGetErrorString(e);
+            return SDPA_ERR_NO_MEMORY;
+        }
+        w.n_counters = want;
+    }
     *out = w.ptr;
+    *counters = w.counters;
     return SDPA_OK;
 }
 
@@ -292,23 +313,26 @@ extern "C" int sdpa_forward(const void* q, const void* k, const void* v, void* o
         if ((st = check_plan(plan, dev)) != SDPA_OK) return reject(st);
         p.splits = plan.splits;
         p.keys_per_split = plan.keys_per_split;
+        int* counters = nullptr;
         if (p.splits > 1) {
             const int64_t rows = B * Hq * Lq;
             const size_t o_bytes = (size_t)rows * p.splits * Dv * sizeof(float);
             const size_t l_bytes = (size_t)rows * p.splits * sizeof(float);
+            const size_t n_cnt = mma ? decode_mma_counters(p, plan) : 0;
             void* ws = nullptr;
-            if ((st = workspace(dev.device, stream, o_bytes + l_bytes + 256, &ws)) != SDPA_OK) return reject(st);
+            if ((st = workspace(dev.device, stream, o_bytes + l_bytes + 256, n_cnt, &ws, &counters)) != SDPA_OK)
+                return reject(st);
             p.part_o = reinterpret_cast<float*>(ws);
             p.part_lse = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + ((o_bytes + 255) / 256) * 256);
         }
         if (log) log_once(mma ? "decode_mma" : "decode_ffma", p, dtype, plan);
         e = timed(mma ? SDPA_KERNEL_DECODE_MMA : SDPA_KERNEL_DECODE_FFMA, stream, [&] {
-            return mma ? decode_mma_launch(p, dtype, plan, stream) : ffma_launch(p, dtype, plan, stream);
+            return mma ? decode_mma_launch(p, dtype, plan, counters, stream) : ffma_launch(p, dtype, plan, stream);
         });
         if (e != cudaSuccess) return cuda_fail(e);
         (mma ? c_dmma : c_dffma).fetch_add(1, std::memory_order_relaxed);
         launches = 1;
-        if (p.splits > 1) {
+        if (p.splits > 1 && !mma) {   // the mma decode kernel merges its splits itself
             if ((e = timed(SDPA_KERNEL_COMBINE, stream, [&] { return combine_launch(p, dtype, stream); })) !=
                 cudaSuccess)
                 return cuda_fail(e);
@@ -392,11 +416,12 @@ extern "C" int sdpa_check_device_error(void* stream_ptr, int* code_out) {
 extern "C" int sdpa_shutdown(void) {
     std::lock_guard<std::mutex> lk(g_mu);
     for (auto& kv : g_ws) {
-        if (kv.second.ptr) {
+        if (kv.second.ptr || kv.second.counters) {
             int cur = 0;
             cudaGetDevice(&cur);
             cudaSetDevice(kv.first.first);
             cudaFree(kv.second.ptr);   // synchronous: the owning stream may no longer exist
+            if (kv.second.counters) cudaFree(kv.second.counters);
             cudaSetDevice(cur);
         }
     }

@@ -45,6 +45,45 @@ __device__ __forceinline__ float fast_exp2(float x) {  // 2^x on the MUFU unit; 
     return y;
 }
 
+// ------------------------------------------------------------------ packed fp32 pairs (f32x2)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ uint64_t f2_bits(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for both halves on the FMA and integer pipes (no MUFU).  Range reduction
+// n = round(x) through the float magic number 1.5 * 2^23, f = x - n in
+// [-1/2, 1/2], cubic p(f) ~ 2^f (least-squares fit in relative error,
+// exp2_poly_fit.py; max relative error 1.4e-4 over [-120, 8]), n added to the
+// exponent field.  Inputs are clamped at -126, so -inf gives ~1e-38, not 0:
+// callers use it only where no key is masked.
+__device__ __forceinline__ uint64_t f2_exp2_poly(uint64_t x) {
+    constexpr float kMagic = 12582912.0f;
+    constexpr uint32_t kMagicShifted = 0x4B400000u << 23;
+    const uint64_t xc = f2_pack(fmaxf(f2_lo(x), -126.f), fmaxf(f2_hi(x), -126.f));
+    const uint64_t t = f2_add(xc, f2_pack(kMagic, kMagic));
+    const uint64_t n = f2_add(t, f2_pack(-kMagic, -kMagic));
+    const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);
+    uint64_t q = f2_fma(f, f2_pack(5.502926558e-02f, 5.502926558e-02f), f2_pack(2.422569841e-01f, 2.422569841e-01f));
+    q = f2_fma(q, f, f2_pack(6.932530403e-01f, 6.932530403e-01f));
+    q = f2_fma(q, f, f2_pack(9.999513626e-01f, 9.999513626e-01f));
+    const uint32_t r0 = (uint32_t)q + ((uint32_t)t << 23) - kMagicShifted;
+    const uint32_t r1 = (uint32_t)(q >> 32) + ((uint32_t)(t >> 32) << 23) - kMagicShifted;
+    return f2_bits(r0, r1);
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -120,16 +159,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
     return ok != 0;
 }
-// Bounded wait: gives up after `limit` polls, records `code` in the device error
-// flag and returns false.  No wait in this library can spin forever.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int code,
-                                                  uint32_t limit = (1u << 26)) {
-    for (uint32_t it = 0; it < limit; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-    }
-    atomicCAS(&g_sdpa_device_error, 0, code);
-    return false;
-}
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
 }
@@ -144,6 +173,36 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, uint
         "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
         : "memory");
 }
+// Tile load through a map built by make_tensor_map: coordinates by role.
+__device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, uint64_t* bar, const MapAxes& ax,
+                                         int d0, int l, int h, int b) {
+    int c[4] = {d0, 0, 0, 0};
+    if (ax.l_pos) c[ax.l_pos] = l;
+    if (ax.h_pos) c[ax.h_pos] = h;
+    if (ax.b_pos) c[ax.b_pos] = b;
+    tma_load_4d(dst, map, bar, c[0], c[1], c[2], c[3]);
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait on an mbarrier phase: about 2 s, then the device error flag is
+// set and false returned.  No wait in this library can spin forever.
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int code) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer() - t0 > 2000000000ull) {
+            atomicCAS(&g_sdpa_device_error, 0, code);
+            return false;
+        }
+    }
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(tmap) : "memory");
 }

@@ -2,6 +2,7 @@
 // kernel translation units.  Not part of the public ABI (include/sdpa.h is).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -61,15 +62,34 @@ struct DeviceInfo {
     int cc_major, cc_minor;
 };
 
+// Which tensor-map dimension carries the sequence, head and batch index
+// (the host orders the three by stride); pos 0 means "always coordinate 0".
+struct MapAxes {
+    int l_pos, h_pos, b_pos;
+};
+
+// A 4-D tiled TMA map of a 16-bit tensor given by (b, h, l, d) element strides
+// `st`: dim 0 = d (extent D), then the sequence / head / batch axes ordered by
+// stride (an extent-1 or zero-stride axis is pinned to coordinate 0); box =
+// 64 elements x box_rows sequence rows; 128-byte swizzle; zero fill out of
+// bounds.  tma_map.cu.
+bool make_tensor_map(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L, int64_t H,
+                     int64_t B, const int64_t* st, int box_rows);
+
 // ---- fp32 (and generic) flash kernel on CUDA cores: flash_ffma.cu
 bool ffma_supported(int dtype, int64_t Dqk, int64_t Dv);
 LaunchPlan ffma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev, bool split_keys);
 cudaError_t ffma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, cudaStream_t stream);
 
-// ---- fp16/bf16 split-K decode on mma.sync: decode_mma.cu
+// ---- fp16/bf16 split-K decode (TMA + mma.sync, combine fused): decode_mma.cu
+// With plan.splits > 1 the kernel needs p.part_o / p.part_lse and
+// decode_mma_counters(p, plan) ints of `counters` that are zero on entry (the
+// kernel leaves them zero again).
 bool decode_mma_supported(int dtype, int64_t Dqk, int64_t Dv);
 LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev);
-cudaError_t decode_mma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, cudaStream_t stream);
+size_t decode_mma_counters(const AttnParams& p, const LaunchPlan& plan);
+cudaError_t decode_mma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, int* counters,
+                              cudaStream_t stream);
 
 // ---- log-sum-exp combine of split-K partials + zero fill: combine.cu
 cudaError_t combine_launch(const AttnParams& p, int dtype, cudaStream_t stream);

@@ -20,8 +20,11 @@
 // receive that address.  Make that first call before any stream capture.
 //
 // Every call on a device shares the one array and leaves the last call's
-// partials in it.  Nothing in it must start at zero: each split writes all of
-// its partials before the combine kernel reads them.  Calls that can overlap
+// partials in it.  Its first kCounterBytes hold the decode kernel's per-group
+// completion counters, which must be zero when the kernel starts: each call
+// clears the ones it uses (cudaMemsetAsync on the call's stream; no
+// allocation) before launching.  Partials need no clearing: each split writes
+// all of its partials before the last CTA reads them.  Calls that can overlap
 // on the GPU (different streams, no ordering between them) race on the array
 // and must not be issued.
 #include <cuda_runtime.h>
@@ -37,6 +40,7 @@ namespace sdpa {
 namespace {
 
 constexpr size_t kNoallocScratchBytes = size_t(4) << 20;   // 4 MiB per device
+constexpr size_t kCounterBytes = 64 * 1024;                 // completion counters at the front
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
@@ -124,15 +128,20 @@ extern "C" int sdpa_forward_noalloc(const void* q, const void* k, const void* v,
         return SDPA_ERR_LAUNCH_CONFIG;
     p.splits = plan.splits;
     p.keys_per_split = plan.keys_per_split;
+    int* counters = nullptr;
     if (p.splits > 1) {
         const int64_t rows = B * Hq * Lq;
         const size_t o_bytes = ((size_t)rows * p.splits * Dv * sizeof(float) + 255) / 256 * 256;
         const size_t l_bytes = (size_t)rows * p.splits * sizeof(float);
-        if (o_bytes + l_bytes > kNoallocScratchBytes) return SDPA_ERR_TOO_LARGE;   // scratch would overflow
-        p.part_o = reinterpret_cast<float*>(nd.scratch);
-        p.part_lse = reinterpret_cast<float*>(reinterpret_cast<char*>(nd.scratch) + o_bytes);
+        const size_t c_bytes = decode_mma_counters(p, plan) * sizeof(int);
+        if (c_bytes > kCounterBytes || kCounterBytes + o_bytes + l_bytes > kNoallocScratchBytes)
+            return SDPA_ERR_TOO_LARGE;   // the scratch array would overflow
+        char* base = reinterpret_cast<char*>(nd.scratch);
+        counters = reinterpret_cast<int*>(base);
+        p.part_o = reinterpret_cast<float*>(base + kCounterBytes);
+        p.part_lse = reinterpret_cast<float*>(base + kCounterBytes + o_bytes);
+        if (cudaMemsetAsync(counters, 0, c_bytes, stream) != cudaSuccess) return SDPA_ERR_CUDA;
     }
-    if (decode_mma_launch(p, dtype, plan, stream) != cudaSuccess) return SDPA_ERR_CUDA;
-    if (p.splits > 1 && combine_launch(p, dtype, stream) != cudaSuccess) return SDPA_ERR_CUDA;
+    if (decode_mma_launch(p, dtype, plan, counters, stream) != cudaSuccess) return SDPA_ERR_CUDA;
     return SDPA_OK;
 }

@@ -32,7 +32,6 @@
 // Every mbarrier wait is bounded (globaltimer); on expiry the kernel records
 // an error code, drains its TMA loads and MMAs, frees TMEM and exits.
 #include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdlib.h>
@@ -75,45 +74,11 @@ struct TcCfg {
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-// Which tensor-map dimension carries the sequence, head and batch index
-// (the host orders the three by stride); pos 0 means "always coordinate 0".
-struct MapAxes {
-    int l_pos, h_pos, b_pos;
-};
-
 struct TcParams {
     AttnParams p;
     MapAxes q_ax, k_ax, v_ax;
     int q_tiles;
 };
-
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Bounded wait on an mbarrier phase: ~2 s, then the error flag and false.
-__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int code) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer() - t0 > 2000000000ull) {
-            atomicCAS(&g_sdpa_device_error, 0, code);
-            return false;
-        }
-    }
-}
-
-__device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, uint64_t* bar, const MapAxes& ax,
-                                         int d0, int l, int h, int b) {
-    int c[4] = {d0, 0, 0, 0};
-    if (ax.l_pos) c[ax.l_pos] = l;
-    if (ax.h_pos) c[ax.h_pos] = h;
-    if (ax.b_pos) c[ax.b_pos] = b;
-    tma_load_4d(dst, map, bar, c[0], c[1], c[2], c[3]);
-}
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&o)[16]) {
     asm volatile(
@@ -123,7 +88,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&o)[16]) {
         : "r"(taddr));
 }
 
-template <typename T, int DQK, int DVC, int NSLOT, int SPLIT>
+template <typename T, int DQK, int DVC, int NSLOT, int SPLIT, int MASK>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const TcParams tp) {
@@ -151,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // causal work is heaviest for the last query tiles: run them first
     const int tile_idx = (int)blockIdx.x / SPLIT;
     const int half = (int)blockIdx.x % SPLIT;
-    const int qt = (p.mask_kind == 3) ? (tp.q_tiles - 1 - tile_idx) : tile_idx;
+    const int qt = (MASK == 3) ? (tp.q_tiles - 1 - tile_idx) : tile_idx;
     const int hq = blockIdx.y, b = blockIdx.z;
     const int hkv = hq / p.group;
     const int64_t q0 = (int64_t)qt * kBM;
@@ -159,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // number of key tiles this query tile needs (causal: up to the diagonal)
     int64_t kv_len = p.Lk;
-    if (p.mask_kind == 3) {
+    if (MASK == 3) {
         const int64_t last = q0 + kBM - 1 + p.Lk - p.Lq;   // last key that row q0+127 sees
         kv_len = last < 0 ? 0 : (last + 1 < p.Lk ? last + 1 : p.Lk);
     }
@@ -296,6 +261,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const T* mask_t = reinterpret_cast<const T*>(p.mask);
         const uint8_t* mask_b = reinterpret_cast<const uint8_t*>(p.mask);
         const int64_t mrow = (int64_t)b * p.sm[0] + (int64_t)hq * p.sm[1] + i * p.sm[2];
+        const float sc = p.scale_log2;
+        const bool pos_scale = sc > 0.f;
 
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
@@ -310,24 +277,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(tmem + lane_off + buf * kBN + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
             tmem_wait_ld();
 
+            // keys of this tile that row i may see: [0, vis) (sequence end, causal limit)
             const int64_t kbase = (int64_t)j * kBN;
-            float mloc = -INFINITY;
+            int64_t lim = p.Lk - kbase;
+            if (MASK == 3) lim = min(lim, causal_lim - kbase + 1);
+            const int vis = row_ok ? (int)max((int64_t)0, min(lim, (int64_t)kBN)) : 0;
+            const bool partial = __any_sync(0xffffffffu, vis < kBN);   // some key of the tile is hidden
+            // values are left raw where possible and scaled inside the exp's FFMA
+            float mul = sc;
+            if (MASK == 1 || MASK == 2 || !pos_scale) {
+                mul = 1.f;
+                const T* mt_row = mask_t + mrow + kbase * p.sm[3];
+                const uint8_t* mb_row = mask_b + mrow + kbase * p.sm[3];
 #pragma unroll
-            for (int c = 0; c < kBN; ++c) {
-                const int64_t key = kbase + c;
-                float x = __uint_as_float(sr[c]) * p.scale_log2;
-                bool keep = row_ok && key < p.Lk;
-                if (p.mask_kind == 3) {
-                    keep = keep && key <= causal_lim;
-                } else if (p.mask_kind == 1) {
-                    if (keep) x += Elem<T>::to_float(mask_t[mrow + key * p.sm[3]]) * log2e;
-                } else if (p.mask_kind == 2) {
-                    keep = keep && mask_b[mrow + key * p.sm[3]] != 0;
+                for (int c = 0; c < kBN; ++c) {
+                    float x = __uint_as_float(sr[c]) * sc;
+                    bool keep = c < vis;
+                    if (MASK == 1 && keep) x += Elem<T>::to_float(mt_row[(int64_t)c * p.sm[3]]) * log2e;
+                    if (MASK == 2 && keep) keep = mb_row[(int64_t)c * p.sm[3]] != 0;
+                    sr[c] = __float_as_uint(keep ? x : -INFINITY);
                 }
-                x = keep ? x : -INFINITY;
-                sr[c] = __float_as_uint(x);
-                mloc = fmaxf(mloc, x);
+            } else if (partial) {
+#pragma unroll
+                for (int c = 0; c < kBN; ++c) sr[c] = (c < vis) ? sr[c] : __float_as_uint(-INFINITY);
             }
+            float mx8[8];   // eight independent chains instead of one 128-deep chain
+#pragma unroll
+            for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(sr[u]);
+#pragma unroll
+            for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+            const float mloc =
+                fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                      fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * mul;   // scaled max
             const float m_new = fmaxf(m_ref, mloc);
             float alpha = 1.f;
             bool rescale = false;
@@ -338,14 +319,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
             l *= alpha;
+            // p = 2^(s * mul - m) on pairs (f32x2); where no key of the tile is hidden,
+            // one pair in four takes the polynomial on the FMA pipe instead of MUFU
             uint32_t pr[kBN / 2];
+            const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(-m_use, -m_use);
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // four independent sum chains
+            if ((MASK == 0 || MASK == 3) && !partial) {
 #pragma unroll
-            for (int c = 0; c < kBN / 2; ++c) {
-                const float p0 = fast_exp2(__uint_as_float(sr[2 * c]) - m_use);
-                const float p1 = fast_exp2(__uint_as_float(sr[2 * c + 1]) - m_use);
-                l += p0 + p1;
-                pr[c] = pack2<T>(p0, p1);
+                for (int c = 0; c < kBN / 2; ++c) {
+                    const uint64_t x = f2_fma(f2_bits(sr[2 * c], sr[2 * c + 1]), mul2, negm2);
+                    const uint64_t pp = ((c & 3) == 3) ? f2_exp2_poly(x)
+                                                        : f2_pack(fast_exp2(f2_lo(x)), fast_exp2(f2_hi(x)));
+                    acc[c & 3] = f2_add(acc[c & 3], pp);
+                    pr[c] = pack2<T>(f2_lo(pp), f2_hi(pp));
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < kBN / 2; ++c) {
+                    const uint64_t x = f2_fma(f2_bits(sr[2 * c], sr[2 * c + 1]), mul2, negm2);
+                    const uint64_t pp = f2_pack(fast_exp2(f2_lo(x)), fast_exp2(f2_hi(x)));
+                    acc[c & 3] = f2_add(acc[c & 3], pp);
+                    pr[c] = pack2<T>(f2_lo(pp), f2_hi(pp));
+                }
             }
+            const uint64_t acc2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+            l += f2_lo(acc2) + f2_hi(acc2);
 #pragma unroll
             for (int c = 0; c < kBN / 64; ++c)
                 tmem_st32(tmem + lane_off + buf * kBN + c * 32, *reinterpret_cast<uint32_t(*)[32]>(pr + c * 32));
@@ -411,73 +409,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
-// A 4-D tiled map (d, then the sequence / head / batch axes in increasing
-// stride order; an axis of extent 1 or stride 0 is pinned to coordinate 0),
-// 128-byte swizzle, box = 64 elements x box_rows rows, zero fill out of bounds.
-bool make_map(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L, int64_t H,
-              int64_t B, const int64_t* st, int box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    const int64_t esz = 2;
-    struct Axis {
-        int which;   // 0 = l, 1 = h, 2 = b
-        int64_t ext, stride;
-    } axes[3] = {{0, L, st[2] * esz}, {1, H, st[1] * esz}, {2, B, st[0] * esz}};
-    // degenerate axes go last with a stride past every other axis
-    int64_t span = ((D * esz + 15) / 16) * 16;
-    for (auto& a : axes)
-        if (a.ext > 1 && a.stride > 0 && a.stride * a.ext > span) span = a.stride * a.ext;
-    for (auto& a : axes)
-        if (a.ext <= 1 || a.stride == 0) {
-            a.ext = 1;
-            a.stride = ((span + 15) / 16) * 16;
-        }
-    // the sequence axis must stay a real dimension for the box rows; sort by (degenerate, stride)
-    for (int x = 0; x < 3; ++x)
-        for (int y = x + 1; y < 3; ++y) {
-            const bool dx = axes[x].ext == 1 && axes[x].which != 0, dy = axes[y].ext == 1 && axes[y].which != 0;
-            if (dx > dy || (dx == dy && axes[y].stride < axes[x].stride)) {
-                Axis t = axes[x];
-                axes[x] = axes[y];
-                axes[y] = t;
-            }
-        }
-    cuuint64_t gdim[4] = {(cuuint64_t)D, 0, 0, 0};
-    cuuint64_t gstride[3];
-    int pos[3] = {0, 0, 0};
-    for (int x = 0; x < 3; ++x) {
-        gdim[x + 1] = (cuuint64_t)axes[x].ext;
-        gstride[x] = (cuuint64_t)axes[x].stride;
-        pos[axes[x].which] = (axes[x].ext > 1 || axes[x].which == 0) ? x + 1 : 0;
-    }
-    cuuint32_t box[4] = {64, 1, 1, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    for (int x = 0; x < 3; ++x)
-        if (axes[x].which == 0) box[x + 1] = (cuuint32_t)box_rows;
-    const CUtensorMapDataType dt =
-        dtype == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    CUresult r = fn(map, dt, 4, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    ax->l_pos = pos[0];
-    ax->h_pos = pos[1];
-    ax->b_pos = pos[2];
-    return r == CUDA_SUCCESS;
-}
-
 struct Variant {
     int split, smem;
 };
@@ -508,14 +439,26 @@ Variant pick(int64_t Dqk, int64_t Dv) {
     }
 }
 
-template <typename T, int DQK, int DVC, int NSLOT, int SPLIT>
-cudaError_t launch_one(const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const LaunchPlan& plan, cudaStream_t stream) {
-    auto kern = prefill_tc_kernel<T, DQK, DVC, NSLOT, SPLIT>;
+template <typename T, int DQK, int DVC, int NSLOT, int SPLIT, int MASK>
+cudaError_t launch_mask(const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const LaunchPlan& plan, cudaStream_t stream) {
+    auto kern = prefill_tc_kernel<T, DQK, DVC, NSLOT, SPLIT, MASK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
     if (e != cudaSuccess) return e;
     kern<<<plan.grid, plan.block, plan.smem_bytes, stream>>>(mq, mk, mv, tp);
     return cudaGetLastError();
+}
+
+template <typename T, int DQK, int DVC, int NSLOT, int SPLIT>
+cudaError_t launch_one(const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const LaunchPlan& plan, cudaStream_t stream) {
+    switch (tp.p.mask_kind) {
+        case 0: return launch_mask<T, DQK, DVC, NSLOT, SPLIT, 0>(tp, mq, mk, mv, plan, stream);
+        case 1: return launch_mask<T, DQK, DVC, NSLOT, SPLIT, 1>(tp, mq, mk, mv, plan, stream);
+        case 2: return launch_mask<T, DQK, DVC, NSLOT, SPLIT, 2>(tp, mq, mk, mv, plan, stream);
+        case 3: return launch_mask<T, DQK, DVC, NSLOT, SPLIT, 3>(tp, mq, mk, mv, plan, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 template <typename T>
@@ -560,9 +503,9 @@ cudaError_t prefill_tc_launch(const AttnParams& p, int dtype, const LaunchPlan& 
     tp.p = p;
     tp.q_tiles = plan.aux;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, &tp.q_ax, p.q, dtype, p.Dqk, p.Lq, p.Hq, p.B, p.sq, kBM) ||
-        !make_map(&mk, &tp.k_ax, p.k, dtype, p.Dqk, p.Lk, p.Hkv, p.B, p.sk, kBN) ||
-        !make_map(&mv, &tp.v_ax, p.v, dtype, p.Dv, p.Lk, p.Hkv, p.B, p.sv, kBN))
+    if (!make_tensor_map(&mq, &tp.q_ax, p.q, dtype, p.Dqk, p.Lq, p.Hq, p.B, p.sq, kBM) ||
+        !make_tensor_map(&mk, &tp.k_ax, p.k, dtype, p.Dqk, p.Lk, p.Hkv, p.B, p.sk, kBN) ||
+        !make_tensor_map(&mv, &tp.v_ax, p.v, dtype, p.Dv, p.Lk, p.Hkv, p.B, p.sv, kBN))
         return cudaErrorInvalidValue;
     if (dtype == 2) return launch_typed<__nv_bfloat16>(tp, mq, mk, mv, plan, stream);
     return launch_typed<__half>(tp, mq, mk, mv, plan, stream);

@@ -1,0 +1,85 @@
+// tma_map.cu -- host-side construction of TMA tensor maps from explicit
+// (b, h, l, d) element strides (cuTensorMapEncodeTiled through the runtime's
+// driver entry point, so the library links no driver library).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "kernels.h"
+
+namespace sdpa {
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+}  // namespace
+
+// A 4-D tiled map (d, then the sequence / head / batch axes in increasing
+// stride order; an axis of extent 1 or stride 0 is pinned to coordinate 0),
+// 128-byte swizzle, box = 64 elements x box_rows rows, zero fill out of bounds.
+bool make_tensor_map(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L, int64_t H,
+              int64_t B, const int64_t* st, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const int64_t esz = 2;
+    struct Axis {
+        int which;   // 0 = l, 1 = h, 2 = b
+        int64_t ext, stride;
+    } axes[3] = {{0, L, st[2] * esz}, {1, H, st[1] * esz}, {2, B, st[0] * esz}};
+    // degenerate axes go last with a stride past every other axis
+    int64_t span = ((D * esz + 15) / 16) * 16;
+    for (auto& a : axes)
+        if (a.ext > 1 && a.stride > 0 && a.stride * a.ext > span) span = a.stride * a.ext;
+    for (auto& a : axes)
+        if (a.ext <= 1 || a.stride == 0) {
+            a.ext = 1;
+            a.stride = ((span + 15) / 16) * 16;
+        }
+    // the sequence axis must stay a real dimension for the box rows; sort by (degenerate, stride)
+    for (int x = 0; x < 3; ++x)
+        for (int y = x + 1; y < 3; ++y) {
+            const bool dx = axes[x].ext == 1 && axes[x].which != 0, dy = axes[y].ext == 1 && axes[y].which != 0;
+            if (dx > dy || (dx == dy && axes[y].stride < axes[x].stride)) {
+                Axis t = axes[x];
+                axes[x] = axes[y];
+                axes[y] = t;
+            }
+        }
+    cuuint64_t gdim[4] = {(cuuint64_t)D, 0, 0, 0};
+    cuuint64_t gstride[3];
+    int pos[3] = {0, 0, 0};
+    for (int x = 0; x < 3; ++x) {
+        gdim[x + 1] = (cuuint64_t)axes[x].ext;
+        gstride[x] = (cuuint64_t)axes[x].stride;
+        pos[axes[x].which] = (axes[x].ext > 1 || axes[x].which == 0) ? x + 1 : 0;
+    }
+    cuuint32_t box[4] = {64, 1, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    for (int x = 0; x < 3; ++x)
+        if (axes[x].which == 0) box[x + 1] = (cuuint32_t)box_rows;
+    const CUtensorMapDataType dt =
+        dtype == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r = fn(map, dt, 4, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    ax->l_pos = pos[0];
+    ax->h_pos = pos[1];
+    ax->b_pos = pos[2];
+    return r == CUDA_SUCCESS;
+}
+
+
+}  // namespace sdpa

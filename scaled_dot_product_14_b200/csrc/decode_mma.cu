@@ -106,11 +106,12 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         }
         fence_barrier_init();
     }
-    // ---- Q rows of this CTA (zero rows past the group and zero pad columns)
-    {
+    __syncthreads();   // barriers initialised; the producer starts streaming K/V right away
+    if (warp > 0) {
+        // ---- Q rows of this CTA (zero rows past the group and zero pad columns), consumer warps only
         const T* qg = reinterpret_cast<const T*>(p.q);
         constexpr int CH = C::DQKP / 8;   // 16-byte chunks per padded row
-        for (int idx = tid; idx < C::ROWS * CH; idx += C::THREADS) {
+        for (int idx = tid - 32; idx < C::ROWS * CH; idx += C::THREADS - 32) {
             const int r = idx / CH, c = idx % CH;
             const int64_t gr = row0 + r;
             uint4 val = make_uint4(0, 0, 0, 0);
@@ -120,8 +121,8 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
             }
             *reinterpret_cast<uint4*>(Qs + r * C::QS + c * 8) = val;
         }
+        asm volatile("bar.sync 1, %0;\n" ::"n"(W * 32) : "memory");   // consumer warps only
     }
-    __syncthreads();
 
     // ---- key blocks of this split (16 keys each), cut at the causal horizon
     const int64_t nkb = (p.Lk + 15) / 16;
@@ -226,9 +227,11 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
             const uint32_t vbase = kbase + C::NBK * kChunk;
 
             // S^T[16 keys][8*NT rows] = K_blk . Q^T
-            float s[NT][4];
+            float s[NT][4], s2[NT][4];   // even / odd K steps: two independent MMA chains
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) s[nt][c] = s2[nt][c] = 0.f;
             {
                 const int arow = (mi & 1) * 8 + (lane & 7);
                 const uint32_t b_addr = q_base + (uint32_t)(((lane & 7) * C::QS + ((lane >> 3) & 1) * 8) * 2);
@@ -240,9 +243,16 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                     for (int nt = 0; nt < NT; ++nt) {
                         uint32_t b0, b1;
                         ldmatrix_x2(b_addr + (uint32_t)(nt * 8 * C::QS * 2) + ks * 32, b0, b1);
-                        mma_16816<T>(s[nt], a0, a1, a2, a3, b0, b1);
+                        if (ks & 1)
+                            mma_16816<T>(s2[nt], a0, a1, a2, a3, b0, b1);
+                        else
+                            mma_16816<T>(s[nt], a0, a1, a2, a3, b0, b1);
                     }
                 }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) s[nt][c] += s2[nt][c];
             }
 
             // scale, mask, online softmax (log2 domain).  s[nt][c]: key g8 + 8*(c>>1), row 2*t4 + (c&1)
@@ -411,14 +421,19 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         const float4* po = reinterpret_cast<const float4*>(p.part_o + row * S * DV) + c4;
         const float* wr = weights + r * kMaxSplits;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int s = 0; s < S; ++s) {
-            const float ws = wr[s];
-            const float4 v = __ldcg(po + (int64_t)s * (DV / 4));
-            acc.x = fmaf(ws, v.x, acc.x);
-            acc.y = fmaf(ws, v.y, acc.y);
-            acc.z = fmaf(ws, v.z, acc.z);
-            acc.w = fmaf(ws, v.w, acc.w);
+        for (int s0 = 0; s0 < S; s0 += 16) {   // sixteen independent loads in flight per thread
+            float4 v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                v[u] = (s0 + u < S) ? __ldcg(po + (int64_t)(s0 + u) * (DV / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const float ws = (s0 + u < S) ? wr[s0 + u] : 0.f;
+                acc.x = fmaf(ws, v[u].x, acc.x);
+                acc.y = fmaf(ws, v[u].y, acc.y);
+                acc.z = fmaf(ws, v[u].z, acc.z);
+                acc.w = fmaf(ws, v[u].w, acc.w);
+            }
         }
         const float inv = wr[kMaxSplits - 1];
         T* og = reinterpret_cast<T*>(p.out) + b * p.so[0] + h * p.so[1] + i * p.so[2] + c4 * 4;

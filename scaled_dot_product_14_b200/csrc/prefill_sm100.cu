@@ -88,6 +88,154 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&o)[16]) {
         : "r"(taddr));
 }
 
+
+// ---------------------------------------------------------------- per-row softmax (shared by both kernels)
+// Thread t of a softmax warpgroup owns query row t of its 128-row tile, which
+// is TMEM lane t.  For key tile j it loads that row of S, applies scale, masks
+// and the causal / sequence limits, updates the running max (log2 domain) and
+// sum, and writes P (16-bit pairs) over the first 64 columns of the same S
+// buffer.  The caller rescales O by `alpha` when `rescale` is set, after the
+// previous tile's P V has completed.
+template <typename T, int MASK>
+struct RowSoftmax {
+    float m_ref, l;
+    bool row_ok, pos_scale;
+    float sc;
+    int64_t Lk, causal_lim, mrow, msm3;
+    const T* mask_t;
+    const uint8_t* mask_b;
+
+    __device__ __forceinline__ void init(const AttnParams& p, int64_t b, int64_t hq, int64_t i) {
+        m_ref = -INFINITY;
+        l = 0.f;
+        row_ok = i < p.Lq;
+        sc = p.scale_log2;
+        pos_scale = sc > 0.f;
+        Lk = p.Lk;
+        causal_lim = i + p.Lk - p.Lq;
+        mrow = b * p.sm[0] + hq * p.sm[1] + i * p.sm[2];
+        msm3 = p.sm[3];
+        mask_t = reinterpret_cast<const T*>(p.mask);
+        mask_b = reinterpret_cast<const uint8_t*>(p.mask);
+    }
+
+    __device__ __forceinline__ void tile(uint32_t s_taddr, int64_t kbase, float& alpha, bool& rescale) {
+        const float log2e = 1.4426950408889634f;
+        uint32_t sr[kBN];
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c)
+            tmem_ld32(s_taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
+        tmem_wait_ld();
+
+        // keys of this tile that the row may see: [0, vis) (sequence end, causal limit)
+        int64_t lim = Lk - kbase;
+        if (MASK == 3) lim = min(lim, causal_lim - kbase + 1);
+        const int vis = row_ok ? (int)max((int64_t)0, min(lim, (int64_t)kBN)) : 0;
+        const bool partial = __any_sync(0xffffffffu, vis < kBN);   // some key of the tile is hidden
+        // values stay raw where possible and are scaled inside the exponent's FFMA
+        float mul = sc;
+        if (MASK == 1 || MASK == 2 || !pos_scale) {
+            mul = 1.f;
+            const T* mt_row = mask_t + mrow + kbase * msm3;
+            const uint8_t* mb_row = mask_b + mrow + kbase * msm3;
+#pragma unroll
+            for (int c = 0; c < kBN; ++c) {
+                float x = __uint_as_float(sr[c]) * sc;
+                bool keep = c < vis;
+                if (MASK == 1 && keep) x += Elem<T>::to_float(mt_row[(int64_t)c * msm3]) * log2e;
+                if (MASK == 2 && keep) keep = mb_row[(int64_t)c * msm3] != 0;
+                sr[c] = __float_as_uint(keep ? x : -INFINITY);
+            }
+        } else if (partial) {
+#pragma unroll
+            for (int c = 0; c < kBN; ++c) sr[c] = (c < vis) ? sr[c] : __float_as_uint(-INFINITY);
+        }
+        float mx8[8];   // eight independent chains instead of one 128-deep chain
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(sr[u]);
+#pragma unroll
+        for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+        const float mloc = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * mul;   // scaled max
+        const float m_new = fmaxf(m_ref, mloc);
+        alpha = 1.f;
+        rescale = false;
+        if (m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + kRescaleThreshold)) {
+            rescale = (m_ref != -INFINITY);   // before the first finite max, O holds zeros
+            alpha = rescale ? fast_exp2(m_ref - m_new) : 0.f;
+            m_ref = m_new;
+        }
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        l *= alpha;
+        // p = 2^(s * mul - m) on pairs (f32x2); where no key of the tile is hidden,
+        // one pair in four takes the polynomial on the FMA pipe instead of MUFU.
+        // P goes to TMEM 64 keys at a time.
+        const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(-m_use, -m_use);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // four independent sum chains
+        const bool poly = (MASK == 0 || MASK == 3) && !partial;
+#pragma unroll
+        for (int h = 0; h < kBN / 64; ++h) {
+            uint32_t pr[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                const int e = h * 64 + 2 * c;
+                const uint64_t x = f2_fma(f2_bits(sr[e], sr[e + 1]), mul2, negm2);
+                uint64_t pp;
+                if (poly && (c & 3) == 3)
+                    pp = f2_exp2_poly(x);
+                else
+                    pp = f2_pack(fast_exp2(f2_lo(x)), fast_exp2(f2_hi(x)));
+                acc[c & 3] = f2_add(acc[c & 3], pp);
+                pr[c] = pack2<T>(f2_lo(pp), f2_hi(pp));
+            }
+            tmem_st32(s_taddr + h * 32, pr);
+        }
+        const uint64_t acc2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+        l += f2_lo(acc2) + f2_hi(acc2);
+        tmem_wait_st();
+    }
+};
+
+// O *= f (one row, DVP fp32 columns starting at o_taddr); warp-collective.
+template <int DVP>
+__device__ __forceinline__ void rescale_o(uint32_t o_taddr, float f) {
+#pragma unroll
+    for (int c = 0; c < DVP / 16; ++c) {
+        uint32_t o[16];
+        tmem_ld16(o_taddr + c * 16, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * f);
+        tmem_st16(o_taddr + c * 16, o);
+    }
+    tmem_wait_st();
+}
+
+// out row = O * inv (zeros when `have` is false), converted and stored; warp-collective.
+template <typename T, int DVC, int DVP>
+__device__ __forceinline__ void store_o(uint32_t o_taddr, bool have, float inv, T* og, bool row_ok) {
+#pragma unroll
+    for (int c = 0; c < DVP / 16; ++c) {
+        uint32_t o[16];
+        if (have) {
+            tmem_ld16(o_taddr + c * 16, o);
+            tmem_wait_ld();
+        } else {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) o[u] = 0u;
+        }
+        uint4 w[2];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            wp[u] = pack2<T>(__uint_as_float(o[2 * u]) * inv, __uint_as_float(o[2 * u + 1]) * inv);
+        if (row_ok) {
+            if (c * 16 < DVC) *reinterpret_cast<uint4*>(og + c * 16) = w[0];
+            if (c * 16 + 8 < DVC) *reinterpret_cast<uint4*>(og + c * 16 + 8) = w[1];
+        }
+    }
+}
+
 template <typename T, int DQK, int DVC, int NSLOT, int SPLIT, int MASK>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -254,149 +402,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;   // warps 2,3,4,5 -> TMEM lane quadrants 2,3,0,1
         const int r = quad * 32 + lane;
         const int64_t i = q0 + r;
-        const bool row_ok = i < p.Lq;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const int64_t causal_lim = i + p.Lk - p.Lq;
-        const float log2e = 1.4426950408889634f;
-        const T* mask_t = reinterpret_cast<const T*>(p.mask);
-        const uint8_t* mask_b = reinterpret_cast<const uint8_t*>(p.mask);
-        const int64_t mrow = (int64_t)b * p.sm[0] + (int64_t)hq * p.sm[1] + i * p.sm[2];
-        const float sc = p.scale_log2;
-        const bool pos_scale = sc > 0.f;
-
-        float m_ref = -INFINITY, l = 0.f;
+        RowSoftmax<T, MASK> rs;
+        rs.init(p, b, hq, i);
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
             const int buf = j & 1;
             ok = __all_sync(0xffffffffu, wait_phase(bar_s_full + buf, (j >> 1) & 1, kErrWaitMma));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sr[kBN];
-#pragma unroll
-            for (int c = 0; c < kBN / 32; ++c)
-                tmem_ld32(tmem + lane_off + buf * kBN + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
-            tmem_wait_ld();
-
-            // keys of this tile that row i may see: [0, vis) (sequence end, causal limit)
-            const int64_t kbase = (int64_t)j * kBN;
-            int64_t lim = p.Lk - kbase;
-            if (MASK == 3) lim = min(lim, causal_lim - kbase + 1);
-            const int vis = row_ok ? (int)max((int64_t)0, min(lim, (int64_t)kBN)) : 0;
-            const bool partial = __any_sync(0xffffffffu, vis < kBN);   // some key of the tile is hidden
-            // values are left raw where possible and scaled inside the exp's FFMA
-            float mul = sc;
-            if (MASK == 1 || MASK == 2 || !pos_scale) {
-                mul = 1.f;
-                const T* mt_row = mask_t + mrow + kbase * p.sm[3];
-                const uint8_t* mb_row = mask_b + mrow + kbase * p.sm[3];
-#pragma unroll
-                for (int c = 0; c < kBN; ++c) {
-                    float x = __uint_as_float(sr[c]) * sc;
-                    bool keep = c < vis;
-                    if (MASK == 1 && keep) x += Elem<T>::to_float(mt_row[(int64_t)c * p.sm[3]]) * log2e;
-                    if (MASK == 2 && keep) keep = mb_row[(int64_t)c * p.sm[3]] != 0;
-                    sr[c] = __float_as_uint(keep ? x : -INFINITY);
-                }
-            } else if (partial) {
-#pragma unroll
-                for (int c = 0; c < kBN; ++c) sr[c] = (c < vis) ? sr[c] : __float_as_uint(-INFINITY);
-            }
-            float mx8[8];   // eight independent chains instead of one 128-deep chain
-#pragma unroll
-            for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(sr[u]);
-#pragma unroll
-            for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
-            const float mloc =
-                fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                      fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * mul;   // scaled max
-            const float m_new = fmaxf(m_ref, mloc);
-            float alpha = 1.f;
-            bool rescale = false;
-            if (m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + kRescaleThreshold)) {
-                rescale = (m_ref != -INFINITY);   // before the first finite max, O holds zeros
-                alpha = rescale ? fast_exp2(m_ref - m_new) : 0.f;
-                m_ref = m_new;
-            }
-            const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-            l *= alpha;
-            // p = 2^(s * mul - m) on pairs (f32x2); where no key of the tile is hidden,
-            // one pair in four takes the polynomial on the FMA pipe instead of MUFU
-            uint32_t pr[kBN / 2];
-            const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(-m_use, -m_use);
-            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // four independent sum chains
-            if ((MASK == 0 || MASK == 3) && !partial) {
-#pragma unroll
-                for (int c = 0; c < kBN / 2; ++c) {
-                    const uint64_t x = f2_fma(f2_bits(sr[2 * c], sr[2 * c + 1]), mul2, negm2);
-                    const uint64_t pp = ((c & 3) == 3) ? f2_exp2_poly(x)
-                                                        : f2_pack(fast_exp2(f2_lo(x)), fast_exp2(f2_hi(x)));
-                    acc[c & 3] = f2_add(acc[c & 3], pp);
-                    pr[c] = pack2<T>(f2_lo(pp), f2_hi(pp));
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < kBN / 2; ++c) {
-                    const uint64_t x = f2_fma(f2_bits(sr[2 * c], sr[2 * c + 1]), mul2, negm2);
-                    const uint64_t pp = f2_pack(fast_exp2(f2_lo(x)), fast_exp2(f2_hi(x)));
-                    acc[c & 3] = f2_add(acc[c & 3], pp);
-                    pr[c] = pack2<T>(f2_lo(pp), f2_hi(pp));
-                }
-            }
-            const uint64_t acc2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
-            l += f2_lo(acc2) + f2_hi(acc2);
-#pragma unroll
-            for (int c = 0; c < kBN / 64; ++c)
-                tmem_st32(tmem + lane_off + buf * kBN + c * 32, *reinterpret_cast<uint32_t(*)[32]>(pr + c * 32));
-            tmem_wait_st();
-
+            float alpha;
+            bool rescale;
+            rs.tile(tmem + lane_off + buf * kBN, (int64_t)j * kBN, alpha, rescale);
             if (j > 0) {
                 ok = __all_sync(0xffffffffu, wait_phase(bar_o_done, (j - 1) & 1, kErrWaitMma));
                 if (!ok) break;
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale)) {
-                    const float f = rescale ? alpha : 1.f;
-#pragma unroll
-                    for (int c = 0; c < C::DVP / 16; ++c) {
-                        uint32_t o[16];
-                        tmem_ld16(tmem + lane_off + C::O_COL + c * 16, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int u = 0; u < 16; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * f);
-                        tmem_st16(tmem + lane_off + C::O_COL + c * 16, o);
-                    }
-                    tmem_wait_st();
-                }
+                if (__any_sync(0xffffffffu, rescale)) rescale_o<C::DVP>(tmem + lane_off + C::O_COL, rescale ? alpha : 1.f);
             }
             tc_fence_before();
             mbar_arrive(bar_p_full + buf);
         }
-
         // epilogue: O / l -> dtype, stored through the output strides
         if (ok && n_tiles > 0)
             ok = __all_sync(0xffffffffu, wait_phase(bar_o_done, (n_tiles - 1) & 1, kErrWaitMma));
         tc_fence_after();
         T* og = reinterpret_cast<T*>(p.out) + (int64_t)b * p.so[0] + (int64_t)hq * p.so[1] + i * p.so[2] + dv0;
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
-#pragma unroll
-        for (int c = 0; c < C::DVP / 16; ++c) {
-            uint32_t o[16];
-            if (n_tiles > 0 && ok) {
-                tmem_ld16(tmem + lane_off + C::O_COL + c * 16, o);
-                tmem_wait_ld();
-            } else {
-#pragma unroll
-                for (int u = 0; u < 16; ++u) o[u] = 0u;
-            }
-            uint4 w[2];
-            uint32_t* wp = reinterpret_cast<uint32_t*>(w);
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                wp[u] = pack2<T>(__uint_as_float(o[2 * u]) * inv, __uint_as_float(o[2 * u + 1]) * inv);
-            if (row_ok) {
-                if (c * 16 < DVC) *reinterpret_cast<uint4*>(og + c * 16) = w[0];
-                if (c * 16 + 8 < DVC) *reinterpret_cast<uint4*>(og + c * 16 + 8) = w[1];
-            }
-        }
+        store_o<T, DVC, C::DVP>(tmem + lane_off + C::O_COL, n_tiles > 0 && ok, rs.l > 0.f ? 1.f / rs.l : 0.f, og,
+                                rs.row_ok);
     }
 
     // teardown: every role has drained its asynchronous work
@@ -408,26 +441,258 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+
+// ---------------------------------------------------------------- two query tiles per CTA (ping-pong)
+// For Dv <= 128 per CTA: 256 query rows of one (batch, head) as tiles A and B
+// that share every K/V chunk.  TMEM: S_A [0,128), S_B [128,256), O_A from 256,
+// O_B from 384.  Two softmax warpgroups (warps 2-5: tile A, 6-9: tile B) take
+// turns on the tensor core: while one computes its exponentials the MMA warp
+// runs the other tile's P V and next S.  MMAs issued by one thread execute in
+// order, so S_X(j+1) may be issued right after PV_X(j), which reads P_X(j)
+// from the same TMEM columns.
+constexpr int kThreads2 = 320;   // 10 warps
+
+template <int DQK, int DVC, int NSLOT>
+struct Tc2Cfg {
+    static constexpr int NBQ = cdiv(DQK, 64);
+    static constexpr int NBV = cdiv(DVC, 64);
+    static constexpr int KSTEPS = cdiv(DQK, 16);
+    static constexpr int DVP = cdiv(DVC, 16) * 16;
+    static constexpr int Q_TILE = NBQ * kBM * 128;
+    static constexpr int OFF_RING = 2 * Q_TILE;
+    static constexpr int OFF_BAR = OFF_RING + NSLOT * kChunk;
+    static constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 + 2 + 2 + 1;
+    static constexpr int SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(DVP <= 128, "two O tiles of at most 128 columns");
+    static_assert(NSLOT >= NBQ + NBV + 1, "ring holds K(j+1) and V(j) at once");
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+template <typename T, int DQK, int DVC, int NSLOT, int MASK>
+__global__ void __launch_bounds__(kThreads2, 1)
+    prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const TcParams tp) {
+    using C = Tc2Cfg<DQK, DVC, NSLOT>;
+    constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    const AttnParams& p = tp.p;
+
+    extern __shared__ unsigned char smem_dyn[];
+    unsigned char* smem =
+        reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t ring = s_base + C::OFF_RING;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* bar_q = bars;
+    uint64_t* bar_full = bars + 1;              // [NSLOT]
+    uint64_t* bar_empty = bar_full + NSLOT;     // [NSLOT]
+    uint64_t* bar_s_full = bar_empty + NSLOT;   // [2]: tile A, tile B
+    uint64_t* bar_p_full = bar_s_full + 2;      // [2]
+    uint64_t* bar_o_done = bar_p_full + 2;      // [2]
+    uint64_t* bar_drain = bar_o_done + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int pair = (MASK == 3) ? (tp.q_tiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+    const int hq = blockIdx.y, b = blockIdx.z;
+    const int hkv = hq / p.group;
+    const int64_t q0 = (int64_t)pair * 2 * kBM;   // tile A rows [q0, q0+128), tile B the next 128
+
+    int64_t kv_len = p.Lk;   // keys the pair needs (tile B sees the most under causal masking)
+    if (MASK == 3) {
+        const int64_t last = q0 + 2 * kBM - 1 + p.Lk - p.Lq;
+        kv_len = last < 0 ? 0 : (last + 1 < p.Lk ? last + 1 : p.Lk);
+    }
+    const int n_tiles = (int)((kv_len + kBN - 1) / kBN);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < NSLOT; ++s) {
+            mbar_init(bar_full + s, 1);
+            mbar_init(bar_empty + s, 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar_s_full + s, 1);
+            mbar_init(bar_p_full + s, 128);
+            mbar_init(bar_o_done + s, 1);
+        }
+        mbar_init(bar_drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    constexpr int PER_TILE = C::NBQ + C::NBV;   // ring chunks per key tile: K(j) then V(j)
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer: K(j), V(j), ...
+        if (lane == 0 && n_tiles > 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_arrive_expect_tx(bar_q, 2 * C::Q_TILE);
+            for (int t2 = 0; t2 < 2; ++t2)
+                for (int c = 0; c < C::NBQ; ++c)
+                    tma_load(s_base + t2 * C::Q_TILE + c * kChunk, &tmQ, bar_q, tp.q_ax, c * 64,
+                             (int)(q0 + t2 * kBM), hq, b);
+            int seq = 0;
+            bool ok = true;
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                for (int c = 0; c < PER_TILE && ok; ++c) {
+                    const int slot = seq % NSLOT;
+                    if (!(ok = wait_phase(bar_empty + slot, ((seq / NSLOT) & 1) ^ 1, kErrWaitSlot))) break;
+                    mbar_arrive_expect_tx(bar_full + slot, kChunk);
+                    if (c < C::NBQ)
+                        tma_load(ring + slot * kChunk, &tmK, bar_full + slot, tp.k_ax, c * 64, j * kBN, hkv, b);
+                    else
+                        tma_load(ring + slot * kChunk, &tmV, bar_full + slot, tp.v_ax, (c - C::NBQ) * 64, j * kBN,
+                                 hkv, b);
+                    ++seq;
+                }
+            }
+            if (!ok) {
+                wait_phase(bar_q, 0, kErrWaitTmaLoad);
+                for (int x = (seq > NSLOT ? seq - NSLOT : 0); x < seq; ++x)
+                    wait_phase(bar_full + x % NSLOT, (x / NSLOT) & 1, kErrWaitTmaLoad);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && n_tiles > 0) {
+            constexpr uint32_t idS = umma_idesc_f16(kBF16 ? 1 : 0, kBM, kBN, 0, 0);
+            bool ok = wait_phase(bar_q, 0, kErrWaitTmaLoad);
+            tc_fence_after();
+            // S_X(j) = Q_X K(j)^T; `release` frees K(j)'s chunks afterwards (tile B, the second user)
+            auto issue_s = [&](int x, int j, bool release) -> bool {
+                const uint32_t d = tmem + (uint32_t)(x * kBN);
+#pragma unroll
+                for (int c = 0; c < C::NBQ; ++c) {
+                    const int seq = j * PER_TILE + c;
+                    const int slot = seq % NSLOT;
+                    if (!wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        if (c * 4 + k4 >= C::KSTEPS) break;
+                        const uint64_t da = umma_desc_sw128(s_base + x * C::Q_TILE + c * kChunk + k4 * 32, 16, 1024);
+                        const uint64_t db = umma_desc_sw128(ring + slot * kChunk + k4 * 32, 16, 1024);
+                        umma_ss(d, da, db, idS, (c > 0 || k4 > 0) ? 1u : 0u);
+                    }
+                    if (release) umma_commit(bar_empty + slot);
+                }
+                umma_commit(bar_s_full + x);
+                return true;
+            };
+            // O_X += P_X(j) V(j); `release` frees V(j)'s chunks afterwards (tile B)
+            auto issue_pv = [&](int x, int j, bool release) -> bool {
+                const uint32_t a_tmem = tmem + (uint32_t)(x * kBN);
+                const uint32_t o_col = 2 * kBN + x * 128;
+#pragma unroll
+                for (int c = 0; c < C::NBV; ++c) {
+                    const int seq = j * PER_TILE + C::NBQ + c;
+                    const int slot = seq % NSLOT;
+                    if (!wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
+                    tc_fence_after();
+                    constexpr int kLastN = C::DVP - 64 * (C::NBV - 1);
+                    const uint32_t idPV =
+                        umma_idesc_f16(kBF16 ? 1 : 0, kBM, (c == C::NBV - 1) ? kLastN : 64, 0, 1);
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk) {
+                        const uint64_t db = umma_desc_sw128(ring + slot * kChunk + kk * 2048, kChunk, 1024);
+                        umma_ts(tmem + o_col + c * 64, a_tmem + kk * 8, db, idPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    if (release) umma_commit(bar_empty + slot);
+                }
+                umma_commit(bar_o_done + x);
+                return true;
+            };
+            if (ok) ok = issue_s(0, 0, false);
+            if (ok) ok = issue_s(1, 0, true);
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                for (int x = 0; x < 2 && ok; ++x) {
+                    if (!(ok = wait_phase(bar_p_full + x, j & 1, kErrWaitSoftmax))) break;
+                    tc_fence_after();
+                    if (!(ok = issue_pv(x, j, x == 1))) break;
+                    if (j + 1 < n_tiles && !(ok = issue_s(x, j + 1, x == 1))) break;
+                }
+            }
+            umma_commit(bar_drain);
+            wait_phase(bar_drain, 0, kErrWaitMma);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warpgroups (A: warps 2-5, B: 6-9)
+        const int x = (warp - 2) >> 2;         // tile of this warpgroup
+        const int quad = warp & 3;             // TMEM lane quadrant
+        const int r = quad * 32 + lane;
+        const int64_t i = q0 + x * kBM + r;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t s_taddr = tmem + lane_off + x * kBN;
+        const uint32_t o_taddr = tmem + lane_off + 2 * kBN + x * 128;
+        RowSoftmax<T, MASK> rs;
+        rs.init(p, b, hq, i);
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            ok = __all_sync(0xffffffffu, wait_phase(bar_s_full + x, j & 1, kErrWaitMma));
+            if (!ok) break;
+            tc_fence_after();
+            float alpha;
+            bool rescale;
+            rs.tile(s_taddr, (int64_t)j * kBN, alpha, rescale);
+            if (j > 0) {
+                ok = __all_sync(0xffffffffu, wait_phase(bar_o_done + x, (j - 1) & 1, kErrWaitMma));
+                if (!ok) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, rescale)) rescale_o<C::DVP>(o_taddr, rescale ? alpha : 1.f);
+            }
+            tc_fence_before();
+            mbar_arrive(bar_p_full + x);
+        }
+        if (ok && n_tiles > 0)
+            ok = __all_sync(0xffffffffu, wait_phase(bar_o_done + x, (n_tiles - 1) & 1, kErrWaitMma));
+        tc_fence_after();
+        T* og = reinterpret_cast<T*>(p.out) + (int64_t)b * p.so[0] + (int64_t)hq * p.so[1] + i * p.so[2];
+        store_o<T, DVC, C::DVP>(o_taddr, n_tiles > 0 && ok, rs.l > 0.f ? 1.f / rs.l : 0.f, og, rs.row_ok);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
 // ---------------------------------------------------------------- host side
 struct Variant {
-    int split, smem;
+    int split, smem, pair;   // pair: two query tiles per CTA (ping-pong kernel)
 };
 
 template <int DQK, int DVC, int NSLOT, int SPLIT>
 Variant variant_of() {
-    return Variant{SPLIT, TcCfg<DQK, DVC, NSLOT, SPLIT>::SMEM};
+    return Variant{SPLIT, TcCfg<DQK, DVC, NSLOT, SPLIT>::SMEM, 0};
+}
+template <int DQK, int DVC, int NSLOT>
+Variant variant2_of() {
+    return Variant{1, Tc2Cfg<DQK, DVC, NSLOT>::SMEM, 1};
 }
 
-// Tile shapes per head dim: (Dqk, Dv per CTA, ring slots, CTAs per query tile).
+// One query tile per CTA: (Dqk, Dv, Dv per CTA, ring slots, CTAs per query tile).
 #define SDPA_TC_VARIANTS(X)             \
-    X(64, 64, 64, 8, 1)                 \
-    X(72, 72, 72, 8, 1)                 \
-    X(80, 80, 80, 8, 1)                 \
-    X(96, 96, 96, 8, 1)                 \
-    X(128, 128, 128, 8, 1)              \
-    X(192, 128, 128, 10, 1)             \
     X(256, 256, 256, 10, 1)             \
     X(512, 512, 256, 6, 2)
+// Two query tiles per CTA: (Dqk, Dv, ring slots).
+#define SDPA_TC2_VARIANTS(X)  \
+    X(64, 64, 10)             \
+    X(72, 72, 10)             \
+    X(80, 80, 10)             \
+    X(96, 96, 10)             \
+    X(128, 128, 10)           \
+    X(192, 128, 8)
 
 Variant pick(int64_t Dqk, int64_t Dv) {
     switch (Dqk * 1000 + Dv) {
@@ -435,14 +700,17 @@ Variant pick(int64_t Dqk, int64_t Dv) {
     case DQ * 1000 + DVV: return variant_of<DQ, DVC, NSL, SP>();
         SDPA_TC_VARIANTS(SDPA_TC_PICK)
 #undef SDPA_TC_PICK
-        default: return Variant{0, 0};
+#define SDPA_TC2_PICK(DQ, DVV, NSL) \
+    case DQ * 1000 + DVV: return variant2_of<DQ, DVV, NSL>();
+        SDPA_TC2_VARIANTS(SDPA_TC2_PICK)
+#undef SDPA_TC2_PICK
+        default: return Variant{0, 0, 0};
     }
 }
 
-template <typename T, int DQK, int DVC, int NSLOT, int SPLIT, int MASK>
-cudaError_t launch_mask(const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                        const LaunchPlan& plan, cudaStream_t stream) {
-    auto kern = prefill_tc_kernel<T, DQK, DVC, NSLOT, SPLIT, MASK>;
+template <typename Kern>
+cudaError_t launch_kernel(Kern kern, const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk,
+                          const CUtensorMap& mv, const LaunchPlan& plan, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
     if (e != cudaSuccess) return e;
     kern<<<plan.grid, plan.block, plan.smem_bytes, stream>>>(mq, mk, mv, tp);
@@ -453,10 +721,22 @@ template <typename T, int DQK, int DVC, int NSLOT, int SPLIT>
 cudaError_t launch_one(const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const LaunchPlan& plan, cudaStream_t stream) {
     switch (tp.p.mask_kind) {
-        case 0: return launch_mask<T, DQK, DVC, NSLOT, SPLIT, 0>(tp, mq, mk, mv, plan, stream);
-        case 1: return launch_mask<T, DQK, DVC, NSLOT, SPLIT, 1>(tp, mq, mk, mv, plan, stream);
-        case 2: return launch_mask<T, DQK, DVC, NSLOT, SPLIT, 2>(tp, mq, mk, mv, plan, stream);
-        case 3: return launch_mask<T, DQK, DVC, NSLOT, SPLIT, 3>(tp, mq, mk, mv, plan, stream);
+        case 0: return launch_kernel(prefill_tc_kernel<T, DQK, DVC, NSLOT, SPLIT, 0>, tp, mq, mk, mv, plan, stream);
+        case 1: return launch_kernel(prefill_tc_kernel<T, DQK, DVC, NSLOT, SPLIT, 1>, tp, mq, mk, mv, plan, stream);
+        case 2: return launch_kernel(prefill_tc_kernel<T, DQK, DVC, NSLOT, SPLIT, 2>, tp, mq, mk, mv, plan, stream);
+        case 3: return launch_kernel(prefill_tc_kernel<T, DQK, DVC, NSLOT, SPLIT, 3>, tp, mq, mk, mv, plan, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T, int DQK, int DVC, int NSLOT>
+cudaError_t launch_two(const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const LaunchPlan& plan, cudaStream_t stream) {
+    switch (tp.p.mask_kind) {
+        case 0: return launch_kernel(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 0>, tp, mq, mk, mv, plan, stream);
+        case 1: return launch_kernel(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 1>, tp, mq, mk, mv, plan, stream);
+        case 2: return launch_kernel(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 2>, tp, mq, mk, mv, plan, stream);
+        case 3: return launch_kernel(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 3>, tp, mq, mk, mv, plan, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -469,6 +749,10 @@ cudaError_t launch_typed(const TcParams& tp, const CUtensorMap& mq, const CUtens
     case DQ * 1000 + DVV: return launch_one<T, DQ, DVC, NSL, SP>(tp, mq, mk, mv, plan, s);
         SDPA_TC_VARIANTS(SDPA_TC_LAUNCH)
 #undef SDPA_TC_LAUNCH
+#define SDPA_TC2_LAUNCH(DQ, DVV, NSL) \
+    case DQ * 1000 + DVV: return launch_two<T, DQ, DVV, NSL>(tp, mq, mk, mv, plan, s);
+        SDPA_TC2_VARIANTS(SDPA_TC2_LAUNCH)
+#undef SDPA_TC2_LAUNCH
         default: return cudaErrorInvalidValue;
     }
 }
@@ -486,9 +770,10 @@ LaunchPlan prefill_tc_plan(const AttnParams& p, int dtype, const DeviceInfo& dev
     (void)dev;
     const Variant v = pick(p.Dqk, p.Dv);
     LaunchPlan plan{};
-    const int64_t q_tiles = (p.Lq + kBM - 1) / kBM;
+    const int64_t rows_per_cta = v.pair ? 2 * kBM : kBM;
+    const int64_t q_tiles = (p.Lq + rows_per_cta - 1) / rows_per_cta;
     plan.grid = dim3((unsigned)(q_tiles * v.split), (unsigned)p.Hq, (unsigned)p.B);
-    plan.block = dim3(kThreads);
+    plan.block = dim3(v.pair ? kThreads2 : kThreads);
     // at least 120 KB: one CTA per SM, so a CTA never waits on another CTA's TMEM
     plan.smem_bytes = (size_t)(v.smem > 120 * 1024 ? v.smem : 120 * 1024);
     plan.splits = 1;

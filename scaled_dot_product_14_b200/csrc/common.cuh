@@ -173,14 +173,14 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, uint
         "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
         : "memory");
 }
-// Tile load through a map built by make_tensor_map: coordinates by role.
+// Tile load through a map built by make_tensor_map: coordinates by role
+// (selects, not an indexed array, so the coordinates stay in registers).
 __device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, uint64_t* bar, const MapAxes& ax,
                                          int d0, int l, int h, int b) {
-    int c[4] = {d0, 0, 0, 0};
-    if (ax.l_pos) c[ax.l_pos] = l;
-    if (ax.h_pos) c[ax.h_pos] = h;
-    if (ax.b_pos) c[ax.b_pos] = b;
-    tma_load_4d(dst, map, bar, c[0], c[1], c[2], c[3]);
+    const int c1 = (ax.l_pos == 1 ? l : 0) + (ax.h_pos == 1 ? h : 0) + (ax.b_pos == 1 ? b : 0);
+    const int c2 = (ax.l_pos == 2 ? l : 0) + (ax.h_pos == 2 ? h : 0) + (ax.b_pos == 2 ? b : 0);
+    const int c3 = (ax.l_pos == 3 ? l : 0) + (ax.h_pos == 3 ? h : 0) + (ax.b_pos == 3 ? b : 0);
+    tma_load_4d(dst, map, bar, d0, c1, c2, c3);
 }
 
 __device__ __forceinline__ uint64_t globaltimer() {

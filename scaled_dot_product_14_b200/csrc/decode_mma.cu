@@ -56,7 +56,8 @@ struct DecodeCfg {
     static constexpr int OFF_BAR = OFF_RING + NSLOT * SLOT;
     static constexpr int MS = DVP + 2;           // merge row: DVP outputs, then m, l
     static constexpr int MERGE_FLOATS = W * ROWS * MS;
-    static constexpr int SMEM = OFF_BAR + 2 * NSLOT * 8 + 16 + 1024;
+    static constexpr int OFF_ROWS = OFF_BAR + 2 * NSLOT * 8 + 16;
+    static constexpr int SMEM = OFF_ROWS + 2 * ROWS * 8 + 1024;
     static constexpr int THREADS = (W + 1) * 32;
     static_assert((MERGE_FLOATS + ROWS * kMaxSplits) * 4 <= NSLOT * SLOT, "merge area must fit in the ring");
     static_assert(SMEM <= 232448, "shared memory budget");
@@ -90,6 +91,8 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* bar_empty = bar_full + NSLOT;
     int* s_flag = reinterpret_cast<int*>(bar_empty + NSLOT);
+    int64_t* row_out = reinterpret_cast<int64_t*>(smem + C::OFF_ROWS);     // [ROWS] output element offset
+    int64_t* row_part = row_out + C::ROWS;                                  // [ROWS] partial row index, -1 = none
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g8 = lane >> 2, t4 = lane & 3;   // MMA fragment coordinates
@@ -120,6 +123,17 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                 val = *reinterpret_cast<const uint4*>(qg + b * p.sq[0] + h * p.sq[1] + i * p.sq[2] + c * 8);
             }
             *reinterpret_cast<uint4*>(Qs + r * C::QS + c * 8) = val;
+        }
+        for (int r = tid - 32; r < C::ROWS; r += C::THREADS - 32) {   // per-row output / partial offsets
+            const int64_t gr = row0 + r;
+            if (gr < R) {
+                const int64_t h = hkv * G + gr / p.Lq, i = gr % p.Lq;
+                row_out[r] = b * p.so[0] + h * p.so[1] + i * p.so[2];
+                row_part[r] = ((int64_t)b * p.Hq + h) * p.Lq + i;
+            } else {
+                row_out[r] = 0;
+                row_part[r] = -1;
+            }
         }
         asm volatile("bar.sync 1, %0;\n" ::"n"(W * 32) : "memory");   // consumer warps only
     }
@@ -350,8 +364,8 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     const int S = p.splits;
     for (int idx = tid; idx < C::ROWS * (DV / 2); idx += C::THREADS) {
         const int r = idx / (DV / 2), e = (idx % (DV / 2)) * 2;
-        const int64_t gr = row0 + r;
-        if (gr >= R) continue;
+        const int64_t row = row_part[r];
+        if (row < 0) continue;
         float mmax = -INFINITY;
 #pragma unroll
         for (int w = 0; w < W; ++w) mmax = fmaxf(mmax, merge[((size_t)w * C::ROWS + r) * C::MS + C::DVP]);
@@ -367,12 +381,10 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
             }
         }
         const float inv = (L > 0.f) ? 1.f / L : 0.f;
-        const int64_t h = hkv * G + gr / p.Lq, i = gr % p.Lq;
         if (S == 1) {
-            T* og = reinterpret_cast<T*>(p.out) + b * p.so[0] + h * p.so[1] + i * p.so[2] + e;
+            T* og = reinterpret_cast<T*>(p.out) + row_out[r] + e;
             *reinterpret_cast<uint32_t*>(og) = pack2<T>(o0 * inv, o1 * inv);
         } else {
-            const int64_t row = ((int64_t)b * p.Hq + h) * p.Lq + i;
             float* po = p.part_o + (row * S + split) * DV + e;
             __stcg(reinterpret_cast<float2*>(po), make_float2(o0 * inv, o1 * inv));
             if (e == 0) __stcg(p.part_lse + row * S + split, (L > 0.f) ? mmax + log2f(L) : -INFINITY);
@@ -390,13 +402,8 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     __threadfence();
     for (int idx = tid; idx < C::ROWS * S; idx += C::THREADS) {   // every split's lse, loaded in parallel
         const int r = idx / S, s2 = idx % S;
-        const int64_t gr = row0 + r;
-        float v = -INFINITY;
-        if (gr < R) {
-            const int64_t row = ((int64_t)b * p.Hq + hkv * G + gr / p.Lq) * p.Lq + gr % p.Lq;
-            v = __ldcg(p.part_lse + row * S + s2);
-        }
-        weights[r * kMaxSplits + s2] = v;
+        const int64_t row = row_part[r];
+        weights[r * kMaxSplits + s2] = (row >= 0) ? __ldcg(p.part_lse + row * S + s2) : -INFINITY;
     }
     __syncthreads();
     for (int r = tid; r < C::ROWS; r += C::THREADS) {   // lse -> weights 2^(lse - max), and 1 / sum
@@ -414,10 +421,8 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     __syncthreads();
     for (int idx = tid; idx < C::ROWS * (DV / 4); idx += C::THREADS) {
         const int r = idx / (DV / 4), c4 = idx % (DV / 4);
-        const int64_t gr = row0 + r;
-        if (gr >= R) continue;
-        const int64_t h = hkv * G + gr / p.Lq, i = gr % p.Lq;
-        const int64_t row = ((int64_t)b * p.Hq + h) * p.Lq + i;
+        const int64_t row = row_part[r];
+        if (row < 0) continue;
         const float4* po = reinterpret_cast<const float4*>(p.part_o + row * S * DV) + c4;
         const float* wr = weights + r * kMaxSplits;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -436,7 +441,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
             }
         }
         const float inv = wr[kMaxSplits - 1];
-        T* og = reinterpret_cast<T*>(p.out) + b * p.so[0] + h * p.so[1] + i * p.so[2] + c4 * 4;
+        T* og = reinterpret_cast<T*>(p.out) + row_out[r] + c4 * 4;
         uint2 pk;
         pk.x = pack2<T>(acc.x * inv, acc.y * inv);
         pk.y = pack2<T>(acc.z * inv, acc.w * inv);

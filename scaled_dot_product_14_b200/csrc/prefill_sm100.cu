@@ -54,6 +54,15 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when t
 
 __host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
 
+// True when the NBV chunks of V(j), which start at ring position first + j * per,
+// never wrap around the NSLOT-slot ring: then one MMA with N = Dv can read all of
+// them (consecutive slots are kChunk bytes apart).
+__host__ __device__ constexpr bool v_contiguous(int first, int per, int nslot, int nbv) {
+    for (int j = 0; j < nslot; ++j)
+        if ((first + j * per) % nslot + nbv > nslot) return false;
+    return true;
+}
+
 // DQK: q/k head dim; DVC: value columns this CTA produces (Dv, or Dv/2 when the
 // pair of CTAs splits Dv: head dim 512); NSLOT: ring slots; SPLIT: CTAs per query tile.
 template <int DQK, int DVC, int NSLOT, int SPLIT>
@@ -363,21 +372,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             auto issue_pv = [&](int j) -> bool {   // O += P_j V_j, P_j read from TMEM
                 const uint32_t a_tmem = tmem + (uint32_t)((j & 1) * kBN);
+                // V(j) starts at ring position 2*NBQ + j*(NBQ+NBV)
+                constexpr bool kContig = v_contiguous(2 * C::NBQ, C::NBQ + C::NBV, NSLOT, C::NBV);
+                if (kContig) {   // one MMA per 16 keys covers every value column
+                    const int slot0 = seq % NSLOT;
 #pragma unroll
-                for (int c = 0; c < C::NBV; ++c) {
-                    const int slot = seq % NSLOT;
-                    if (!wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
+                    for (int c = 0; c < C::NBV; ++c)
+                        if (!wait_phase(bar_full + (seq + c) % NSLOT, ((seq + c) / NSLOT) & 1, kErrWaitTmaLoad))
+                            return false;
                     tc_fence_after();
-                    constexpr int kLastN = C::DVP - 64 * (C::NBV - 1);
-                    const uint32_t idPV =
-                        umma_idesc_f16(kBF16 ? 1 : 0, kBM, (c == C::NBV - 1) ? kLastN : 64, 0, 1);
+                    constexpr uint32_t idPV = umma_idesc_f16(kBF16 ? 1 : 0, kBM, C::DVP, 0, 1);
 #pragma unroll
                     for (int kk = 0; kk < kBN / 16; ++kk) {
-                        const uint64_t db = umma_desc_sw128(ring + slot * kChunk + kk * 2048, kChunk, 1024);
-                        umma_ts(tmem + C::O_COL + c * 64, a_tmem + kk * 8, db, idPV, (j > 0 || kk > 0) ? 1u : 0u);
+                        const uint64_t db = umma_desc_sw128(ring + slot0 * kChunk + kk * 2048, kChunk, 1024);
+                        umma_ts(tmem + C::O_COL, a_tmem + kk * 8, db, idPV, (j > 0 || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit(bar_empty + slot);
-                    ++seq;
+#pragma unroll
+                    for (int c = 0; c < C::NBV; ++c) umma_commit(bar_empty + (seq + c) % NSLOT);
+                    seq += C::NBV;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < C::NBV; ++c) {
+                        const int slot = seq % NSLOT;
+                        if (!wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
+                        tc_fence_after();
+                        constexpr int kLastN = C::DVP - 64 * (C::NBV - 1);
+                        const uint32_t idPV =
+                            umma_idesc_f16(kBF16 ? 1 : 0, kBM, (c == C::NBV - 1) ? kLastN : 64, 0, 1);
+#pragma unroll
+                        for (int kk = 0; kk < kBN / 16; ++kk) {
+                            const uint64_t db = umma_desc_sw128(ring + slot * kChunk + kk * 2048, kChunk, 1024);
+                            umma_ts(tmem + C::O_COL + c * 64, a_tmem + kk * 8, db, idPV,
+                                    (j > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(bar_empty + slot);
+                        ++seq;
+                    }
                 }
                 umma_commit(bar_o_done);
                 return true;
@@ -465,7 +495,8 @@ struct Tc2Cfg {
     static constexpr int SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(DVP <= 128, "two O tiles of at most 128 columns");
-    static_assert(NSLOT >= NBQ + NBV + 1, "ring holds K(j+1) and V(j) at once");
+    static_assert(NSLOT >= 2 * (NBQ + NBV), "ring holds K(j+1) and V(j) at once");
+    static_assert(NSLOT % (NBQ + NBV) == 0, "a tile's V chunks occupy consecutive slots");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -592,22 +623,22 @@ __global__ void __launch_bounds__(kThreads2, 1)
             auto issue_pv = [&](int x, int j, bool release) -> bool {
                 const uint32_t a_tmem = tmem + (uint32_t)(x * kBN);
                 const uint32_t o_col = 2 * kBN + x * 128;
+                const int seq0 = j * PER_TILE + C::NBQ;   // V(j)'s chunks are consecutive ring slots
 #pragma unroll
-                for (int c = 0; c < C::NBV; ++c) {
-                    const int seq = j * PER_TILE + C::NBQ + c;
-                    const int slot = seq % NSLOT;
-                    if (!wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
-                    tc_fence_after();
-                    constexpr int kLastN = C::DVP - 64 * (C::NBV - 1);
-                    const uint32_t idPV =
-                        umma_idesc_f16(kBF16 ? 1 : 0, kBM, (c == C::NBV - 1) ? kLastN : 64, 0, 1);
+                for (int c = 0; c < C::NBV; ++c)
+                    if (!wait_phase(bar_full + (seq0 + c) % NSLOT, ((seq0 + c) / NSLOT) & 1, kErrWaitTmaLoad))
+                        return false;
+                tc_fence_after();
+                constexpr uint32_t idPV = umma_idesc_f16(kBF16 ? 1 : 0, kBM, C::DVP, 0, 1);
+                const uint32_t v0 = ring + (seq0 % NSLOT) * kChunk;
 #pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk) {
-                        const uint64_t db = umma_desc_sw128(ring + slot * kChunk + kk * 2048, kChunk, 1024);
-                        umma_ts(tmem + o_col + c * 64, a_tmem + kk * 8, db, idPV, (j > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    if (release) umma_commit(bar_empty + slot);
+                for (int kk = 0; kk < kBN / 16; ++kk) {   // one MMA per 16 keys covers every value column
+                    const uint64_t db = umma_desc_sw128(v0 + kk * 2048, kChunk, 1024);
+                    umma_ts(tmem + o_col, a_tmem + kk * 8, db, idPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
+                if (release)
+#pragma unroll
+                    for (int c = 0; c < C::NBV; ++c) umma_commit(bar_empty + (seq0 + c) % NSLOT);
                 umma_commit(bar_o_done + x);
                 return true;
             };
@@ -683,16 +714,16 @@ Variant variant2_of() {
 
 // One query tile per CTA: (Dqk, Dv, Dv per CTA, ring slots, CTAs per query tile).
 #define SDPA_TC_VARIANTS(X)             \
-    X(256, 256, 256, 10, 1)             \
+    X(192, 128, 128, 10, 1)             \
+    X(256, 256, 256, 8, 1)              \
     X(512, 512, 256, 6, 2)
-// Two query tiles per CTA: (Dqk, Dv, ring slots).
+// Two query tiles per CTA: (Dqk, Dv, ring slots); slots a multiple of the chunks per key tile.
 #define SDPA_TC2_VARIANTS(X)  \
     X(64, 64, 10)             \
-    X(72, 72, 10)             \
-    X(80, 80, 10)             \
-    X(96, 96, 10)             \
-    X(128, 128, 10)           \
-    X(192, 128, 8)
+    X(72, 72, 8)              \
+    X(80, 80, 8)              \
+    X(96, 96, 8)              \
+    X(128, 128, 8)
 
 Variant pick(int64_t Dqk, int64_t Dv) {
     switch (Dqk * 1000 + Dv) {

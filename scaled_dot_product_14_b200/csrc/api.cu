@@ -314,7 +314,7 @@ extern "C" int sdpa_forward(const void* q, const void* k, const void* v, void* o
         p.splits = plan.splits;
         p.keys_per_split = plan.keys_per_split;
         int* counters = nullptr;
-        if (p.splits > 1) {
+        if (p.splits > 1 && !(mma && decode_mma_uses_cluster(plan))) {   // cluster merges need no workspace
             const int64_t rows = B * Hq * Lq;
             const size_t o_bytes = (size_t)rows * p.splits * Dv * sizeof(float);
             const size_t l_bytes = (size_t)rows * p.splits * sizeof(float);

@@ -14,11 +14,13 @@
 //  * keys are split across CTAs (split-K) so that B*Hkv small problems still
 //    fill the 148 SMs in one wave; the split count scales with 1/(B*Hkv) (same
 //    issue: its two-pass kernel starves the grid when n_kv is small);
-//  * one producer thread streams 16-key blocks of K and V with TMA (128-byte
-//    swizzle, zero fill past Lk) into a CTA-wide ring of NSLOT slots, so about
+//  * one producer thread streams 32-key slots of K and V with TMA (128-byte
+//    swizzle, zero fill past Lk; 4 KB boxes, since one thread issuing 2 KB
+//    boxes cannot keep HBM busy) into a CTA-wide ring of NSLOT slots, so about
 //    200 KB are in flight per SM and the consumer warps issue no load
 //    instructions for K and V;
-//  * consumer warp w takes blocks w, w+W, ...; scores are computed transposed,
+//  * consumer warp w takes the 16-key sub-blocks w, w+W, ... of the slots;
+//    scores are computed transposed,
 //    S^T = K Q^T, so the keys fill the 16-row side of the MMA and the few query
 //    rows the 8-column side; P^T reaches the B operand of O^T += V^T P^T with
 //    one movmatrix per 8x8 block;
@@ -30,14 +32,21 @@
 #include <math.h>
 #include <stdlib.h>
 
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace sdpa {
 namespace {
 
-constexpr int kChunk = 16 * 128;      // 16 keys x 64 head-dim elements (128-byte swizzle)
+constexpr int kSK = 32;                 // keys per ring slot (one TMA box of 32 rows x 128 bytes)
+constexpr int kNSUB = kSK / 16;         // 16-key sub-blocks per slot (one consumer warp each)
+constexpr int kChunk = kSK * 128;       // one 64-element column chunk of a slot
 constexpr int kMaxSplits = 256;
+constexpr int kMaxClusterSplits = 16;   // largest (non-portable) cluster
 
 __host__ __device__ constexpr int round16(int x) { return (x + 15) / 16 * 16; }
 __host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -54,12 +63,15 @@ struct DecodeCfg {
     static constexpr int ROWS = 8 * NT;          // query rows per CTA
     static constexpr int OFF_RING = align1k(ROWS * QS * 2);
     static constexpr int OFF_BAR = OFF_RING + NSLOT * SLOT;
-    static constexpr int MS = DVP + 2;           // merge row: DVP outputs, then m, l
+    static constexpr int MS = DVP + 4;           // merge row: DVP outputs, then m, l (16-byte aligned rows)
     static constexpr int MERGE_FLOATS = W * ROWS * MS;
     static constexpr int OFF_ROWS = OFF_BAR + 2 * NSLOT * 8 + 16;
-    static constexpr int SMEM = OFF_ROWS + 2 * ROWS * 8 + 1024;
+    static constexpr int OFF_COEF = OFF_ROWS + 2 * ROWS * 8;   // [ROWS][W + 1]: merge weights, then lse
+    static constexpr int SMEM = OFF_COEF + ROWS * (W + 1) * 4 + 1024;
     static constexpr int THREADS = (W + 1) * 32;
     static_assert((MERGE_FLOATS + ROWS * kMaxSplits) * 4 <= NSLOT * SLOT, "merge area must fit in the ring");
+    static_assert((MERGE_FLOATS + ROWS * DV + ROWS * (kMaxClusterSplits + 1)) * 4 <= NSLOT * SLOT,
+                  "cluster partials must fit in the ring");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -75,7 +87,7 @@ __device__ __forceinline__ uint32_t swz(uint32_t chunk, int row, int u) {
     return chunk + (uint32_t)(row * 128 + ((u ^ (row & 7)) << 4));
 }
 
-template <typename T, int DQK, int DV, int NT, int W, int NSLOT>
+template <typename T, int DQK, int DV, int NT, int W, int NSLOT, bool CLUSTER>
 __global__ void __launch_bounds__((W + 1) * 32, 1)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const DecParams dp) {
@@ -88,6 +100,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     const uint32_t ring = smem_u32(smem + C::OFF_RING);
     float* merge = reinterpret_cast<float*>(smem + C::OFF_RING);   // reused after the key loop
     float* weights = merge + C::MERGE_FLOATS;                       // [ROWS][splits], last CTA only
+    float* cpart = merge + C::MERGE_FLOATS;                         // cluster path: [ROWS][DV] partial
     uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* bar_empty = bar_full + NSLOT;
     int* s_flag = reinterpret_cast<int*>(bar_empty + NSLOT);
@@ -105,7 +118,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     if (tid == 0) {
         for (int s = 0; s < NSLOT; ++s) {
             mbar_init(bar_full + s, 1);
-            mbar_init(bar_empty + s, 1);
+            mbar_init(bar_empty + s, kNSUB);   // each 16-key sub-block's consumer arrives once
         }
         fence_barrier_init();
     }
@@ -138,19 +151,19 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         asm volatile("bar.sync 1, %0;\n" ::"n"(W * 32) : "memory");   // consumer warps only
     }
 
-    // ---- key blocks of this split (16 keys each), cut at the causal horizon
-    const int64_t nkb = (p.Lk + 15) / 16;
-    const int64_t kbps = p.keys_per_split / 16;
-    const int64_t kb_begin = (int64_t)split * kbps;
-    int64_t kb_end = min(nkb, kb_begin + kbps);
+    // ---- slots of this split (kSK keys each), cut at the causal horizon
+    const int64_t nsl = (p.Lk + kSK - 1) / kSK;
+    const int64_t slps = p.keys_per_split / kSK;
+    const int64_t sl_begin = (int64_t)split * slps;
+    int64_t sl_end = min(nsl, sl_begin + slps);
     if (p.mask_kind == 3) {
         int64_t max_i = -1;   // largest query index among this CTA's rows
         for (int r = 0; r < C::ROWS; ++r)
             if (row0 + r < R) max_i = max(max_i, (row0 + r) % p.Lq);
         const int64_t last = max_i + p.Lk - p.Lq;   // last key any row sees
-        kb_end = min(kb_end, last < 0 ? (int64_t)0 : last / 16 + 1);
+        sl_end = min(sl_end, last < 0 ? (int64_t)0 : last / kSK + 1);
     }
-    const int n_blocks = kb_end > kb_begin ? (int)(kb_end - kb_begin) : 0;
+    const int n_slots = sl_end > sl_begin ? (int)(sl_end - sl_begin) : 0;
 
     // per-thread state: rows (nt*8 + 2*t4 + {0,1}); O^T fragments (consumer warps)
     float m_run[NT][2], l_run[NT][2];
@@ -169,16 +182,16 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0 && n_blocks > 0) {
+        if (lane == 0 && n_slots > 0) {
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             int t = 0;
             bool ok = true;
-            for (; t < n_blocks; ++t) {
+            for (; t < n_slots; ++t) {
                 const int slot = t % NSLOT;
                 if (!(ok = wait_phase(bar_empty + slot, ((t / NSLOT) & 1) ^ 1, kErrWaitSlot))) break;
                 mbar_arrive_expect_tx(bar_full + slot, C::SLOT);
-                const int key0 = (int)((kb_begin + t) * 16);
+                const int key0 = (int)((sl_begin + t) * kSK);
                 const uint32_t base = ring + slot * C::SLOT;
 #pragma unroll
                 for (int c = 0; c < C::NBK; ++c)
@@ -209,9 +222,10 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         const float log2e = 1.4426950408889634f;
         const int mi = lane >> 3;   // which 8x8 matrix this lane addresses in an x4 ldmatrix
 
-        for (int t = w; t < n_blocks; t += W) {
+        for (int item = w; item < n_slots * kNSUB; item += W) {
+            const int t = item / kNSUB, u = item % kNSUB;   // slot t, 16-key sub-block u
             const int slot = t % NSLOT;
-            const int64_t kb = kb_begin + t;
+            const int64_t kb = (sl_begin + t) * kNSUB + u;   // global 16-key block index
             // mask values of this block, loaded before waiting for K/V so the two latencies overlap
             float madd[NT][4];
             bool mkeep[NT][4];
@@ -239,6 +253,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
             if (!__all_sync(0xffffffffu, wait_phase(bar_full + slot, (t / NSLOT) & 1, kErrWaitTmaLoad))) break;
             const uint32_t kbase = ring + slot * C::SLOT;
             const uint32_t vbase = kbase + C::NBK * kChunk;
+            const int rsub = u * 16;   // first row of this sub-block inside the slot
 
             // S^T[16 keys][8*NT rows] = K_blk . Q^T
             float s[NT][4], s2[NT][4];   // even / odd K steps: two independent MMA chains
@@ -247,7 +262,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) s[nt][c] = s2[nt][c] = 0.f;
             {
-                const int arow = (mi & 1) * 8 + (lane & 7);
+                const int arow = rsub + (mi & 1) * 8 + (lane & 7);
                 const uint32_t b_addr = q_base + (uint32_t)(((lane & 7) * C::QS + ((lane >> 3) & 1) * 8) * 2);
 #pragma unroll
                 for (int ks = 0; ks < C::DQKP / 16; ++ks) {
@@ -310,7 +325,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
 
             // O^T[DV][rows] += V^T . P^T
             {
-                const int vrow = (mi >> 1) * 8 + (lane & 7);
+                const int vrow = rsub + (mi >> 1) * 8 + (lane & 7);
 #pragma unroll
                 for (int mt = 0; mt < C::DVP / 16; ++mt) {
                     uint32_t a0, a1, a2, a3;
@@ -338,6 +353,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     }
 
     // ---- merge the consumer warps through shared memory (the ring is drained)
+    __syncwarp();   // the producer warp reconverges (its lane 0 ran the TMA loop) before the CTA barrier
     __syncthreads();
     if (warp > 0) {
         float* mw = merge + (size_t)(warp - 1) * C::ROWS * C::MS;
@@ -362,35 +378,104 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     __syncthreads();
 
     const int S = p.splits;
-    for (int idx = tid; idx < C::ROWS * (DV / 2); idx += C::THREADS) {
-        const int r = idx / (DV / 2), e = (idx % (DV / 2)) * 2;
-        const int64_t row = row_part[r];
-        if (row < 0) continue;
+    float* coef = reinterpret_cast<float*>(smem + C::OFF_COEF);   // [ROWS][W + 1]
+    for (int r = tid; r < C::ROWS; r += C::THREADS) {           // per row: weights of the W warps, lse
         float mmax = -INFINITY;
 #pragma unroll
         for (int w = 0; w < W; ++w) mmax = fmaxf(mmax, merge[((size_t)w * C::ROWS + r) * C::MS + C::DVP]);
-        float L = 0.f, o0 = 0.f, o1 = 0.f;
-        if (mmax != -INFINITY) {
+        float f[W], L = 0.f;
 #pragma unroll
-            for (int w = 0; w < W; ++w) {
-                const float* row = merge + ((size_t)w * C::ROWS + r) * C::MS;
-                const float f = fast_exp2(row[C::DVP] - mmax);   // -inf -> 0
-                L += row[C::DVP + 1] * f;
-                o0 += row[e] * f;
-                o1 += row[e + 1] * f;
-            }
+        for (int w = 0; w < W; ++w) {
+            const float* row = merge + ((size_t)w * C::ROWS + r) * C::MS;
+            f[w] = (mmax == -INFINITY) ? 0.f : fast_exp2(row[C::DVP] - mmax);   // -inf -> 0
+            L += row[C::DVP + 1] * f[w];
         }
         const float inv = (L > 0.f) ? 1.f / L : 0.f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) coef[r * (W + 1) + w] = f[w] * inv;
+        coef[r * (W + 1) + W] = (L > 0.f) ? mmax + log2f(L) : -INFINITY;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C::ROWS * (DV / 4); idx += C::THREADS) {
+        const int r = idx / (DV / 4), c4 = idx % (DV / 4);
+        const int64_t row = row_part[r];
+        if (row < 0) continue;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+            const float cw = coef[r * (W + 1) + w];
+            const float4 v = *reinterpret_cast<const float4*>(merge + ((size_t)w * C::ROWS + r) * C::MS + c4 * 4);
+            acc.x = fmaf(cw, v.x, acc.x);
+            acc.y = fmaf(cw, v.y, acc.y);
+            acc.z = fmaf(cw, v.z, acc.z);
+            acc.w = fmaf(cw, v.w, acc.w);
+        }
         if (S == 1) {
-            T* og = reinterpret_cast<T*>(p.out) + row_out[r] + e;
-            *reinterpret_cast<uint32_t*>(og) = pack2<T>(o0 * inv, o1 * inv);
+            uint2 pk;
+            pk.x = pack2<T>(acc.x, acc.y);
+            pk.y = pack2<T>(acc.z, acc.w);
+            *reinterpret_cast<uint2*>(reinterpret_cast<T*>(p.out) + row_out[r] + c4 * 4) = pk;
+        } else if (CLUSTER) {
+            reinterpret_cast<float4*>(cpart)[r * (DV / 4) + c4] = acc;   // kept for the peers
         } else {
-            float* po = p.part_o + (row * S + split) * DV + e;
-            __stcg(reinterpret_cast<float2*>(po), make_float2(o0 * inv, o1 * inv));
-            if (e == 0) __stcg(p.part_lse + row * S + split, (L > 0.f) ? mmax + log2f(L) : -INFINITY);
+            __stcg(reinterpret_cast<float4*>(p.part_o + (row * S + split) * DV) + c4, acc);
+            if (c4 == 0) __stcg(p.part_lse + row * S + split, coef[r * (W + 1) + W]);
         }
     }
     if (S == 1) return;
+
+    if (CLUSTER) {
+        // ---- the S CTAs of this cluster are the S splits of one (batch, KV head, row group):
+        // each reads every peer's partial over distributed shared memory and writes a
+        // slice of the output; no global round trip, no counter.
+        cluster_sync();
+        float* wgt = cpart + C::ROWS * DV;   // [ROWS][kMaxClusterSplits]: split weights, then 1 / sum
+        for (int idx = tid; idx < C::ROWS * S; idx += C::THREADS) {
+            const int r = idx / S, s2 = idx % S;
+            wgt[r * (kMaxClusterSplits + 1) + s2] =
+                dsmem_ld_f32(dsmem_addr(coef + r * (W + 1) + W, (uint32_t)s2));   // lse of split s2
+        }
+        __syncthreads();
+        for (int r = tid; r < C::ROWS; r += C::THREADS) {
+            float* wr = wgt + r * (kMaxClusterSplits + 1);
+            float mx = -INFINITY;
+            for (int s2 = 0; s2 < S; ++s2) mx = fmaxf(mx, wr[s2]);
+            float sum = 0.f;
+            for (int s2 = 0; s2 < S; ++s2) {
+                const float ws = (mx == -INFINITY) ? 0.f : fast_exp2(wr[s2] - mx);   // -inf -> 0
+                wr[s2] = ws;
+                sum += ws;
+            }
+            wr[kMaxClusterSplits] = (sum > 0.f) ? 1.f / sum : 0.f;
+        }
+        __syncthreads();
+        const int rank = (int)cluster_ctarank();
+        for (int idx = rank * C::THREADS + tid; idx < C::ROWS * (DV / 4); idx += S * C::THREADS) {
+            const int r = idx / (DV / 4), c4 = idx % (DV / 4);
+            if (row_part[r] < 0) continue;
+            const float* wr = wgt + r * (kMaxClusterSplits + 1);
+            const uint32_t local = smem_u32(cpart + (r * (DV / 4) + c4) * 4);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+            for (int s2 = 0; s2 < S; ++s2) {
+                uint32_t ra;
+                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local), "r"(s2));
+                const float4 v = dsmem_ld_f32x4(ra);
+                const float ws = wr[s2];
+                acc.x = fmaf(ws, v.x, acc.x);
+                acc.y = fmaf(ws, v.y, acc.y);
+                acc.z = fmaf(ws, v.z, acc.z);
+                acc.w = fmaf(ws, v.w, acc.w);
+            }
+            const float inv = wr[kMaxClusterSplits];
+            uint2 pk;
+            pk.x = pack2<T>(acc.x * inv, acc.y * inv);
+            pk.y = pack2<T>(acc.z * inv, acc.w * inv);
+            *reinterpret_cast<uint2*>(reinterpret_cast<T*>(p.out) + row_out[r] + c4 * 4) = pk;
+        }
+        cluster_sync();   // no CTA leaves while a peer may still read its shared memory
+        return;
+    }
 
     // ---- the last CTA of this (batch, KV head, row group) merges every split
     __threadfence();
@@ -464,14 +549,14 @@ Shape shape_of() {
 // (Dqk, Dv, W, NSLOT) per head dim; NT in {1, 2, 4} with the O^T accumulators at
 // DVP*NT/4 registers per thread (NT = 1 only at Dv = 512, NT <= 2 at Dv = 256).
 #define SDPA_DECODE_DIMS(X) \
-    X(64, 64, 4, 32)        \
-    X(72, 72, 4, 24)        \
-    X(80, 80, 4, 24)        \
-    X(96, 96, 4, 24)        \
-    X(128, 128, 4, 24)      \
-    X(192, 128, 4, 18)      \
-    X(256, 256, 4, 12)      \
-    X(512, 512, 4, 6)
+    X(64, 64, 4, 24)        \
+    X(72, 72, 4, 12)        \
+    X(80, 80, 4, 12)        \
+    X(96, 96, 4, 12)        \
+    X(128, 128, 4, 12)      \
+    X(192, 128, 4, 9)       \
+    X(256, 256, 4, 6)       \
+    X(512, 512, 4, 3)
 
 constexpr int nt_cap(int dv) { return dv >= 512 ? 1 : (dv >= 256 ? 2 : 4); }
 constexpr int nt_fix(int want, int dv) { return want < nt_cap(dv) ? want : nt_cap(dv); }
@@ -492,14 +577,89 @@ Shape pick_shape(int64_t Dqk, int64_t Dv, int64_t rows) {
     }
 }
 
+// Clusters of `splits` CTAs the device can hold at once for this kernel (0 on error).
+template <typename T, int DQK, int DV, int NT, int W, int NS>
+int max_active_clusters(int splits, size_t smem) {
+    auto kern = decode_mma_kernel<T, DQK, DV, NT, W, NS, true>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+        (splits > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)splits);
+    cfg.blockDim = dim3((unsigned)((W + 1) * 32));
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
+int active_clusters(int dtype, int64_t Dqk, int64_t Dv, int nt, int splits, size_t smem) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, int64_t, int64_t, int, int>, int> cache;
+    std::lock_guard<std::mutex> lk(mu);
+    const auto key = std::make_tuple(dtype, Dqk, Dv, nt, splits);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    int n = 0;
+    switch (Dqk * 1000 + Dv) {
+#define SDPA_DECODE_OCC(DQ, DVV, W, NS)                                                                      \
+    case DQ * 1000 + DVV:                                                                                    \
+        if (dtype == 2)                                                                                      \
+            n = nt == 1 ? max_active_clusters<__nv_bfloat16, DQ, DVV, 1, W, NS>(splits, smem)                  \
+                : nt == 2 ? max_active_clusters<__nv_bfloat16, DQ, DVV, nt_fix(2, DVV), W, NS>(splits, smem)   \
+                          : max_active_clusters<__nv_bfloat16, DQ, DVV, nt_fix(4, DVV), W, NS>(splits, smem);  \
+        else                                                                                                 \
+            n = nt == 1 ? max_active_clusters<__half, DQ, DVV, 1, W, NS>(splits, smem)                         \
+                : nt == 2 ? max_active_clusters<__half, DQ, DVV, nt_fix(2, DVV), W, NS>(splits, smem)          \
+                          : max_active_clusters<__half, DQ, DVV, nt_fix(4, DVV), W, NS>(splits, smem);         \
+        break;
+        SDPA_DECODE_DIMS(SDPA_DECODE_OCC)
+#undef SDPA_DECODE_OCC
+        default: n = 0;
+    }
+    cache[key] = n;
+    return n;
+}
+
 template <typename T, int DQK, int DV, int NT, int W, int NS>
 cudaError_t launch_one(const DecParams& dp, const CUtensorMap& mk, const CUtensorMap& mv, const LaunchPlan& plan,
                        cudaStream_t stream) {
-    auto kern = decode_mma_kernel<T, DQK, DV, NT, W, NS>;
+    const bool cluster = plan.cluster > 1;
+    auto kern = cluster ? decode_mma_kernel<T, DQK, DV, NT, W, NS, true> : decode_mma_kernel<T, DQK, DV, NT, W, NS, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
     if (e != cudaSuccess) return e;
-    kern<<<plan.grid, plan.block, plan.smem_bytes, stream>>>(mk, mv, dp);
-    return cudaGetLastError();
+    if (!cluster) {
+        kern<<<plan.grid, plan.block, plan.smem_bytes, stream>>>(mk, mv, dp);
+        return cudaGetLastError();
+    }
+    if (plan.splits > 8 && (e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
+                               cudaSuccess)
+        return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = plan.grid;
+    cfg.blockDim = plan.block;
+    cfg.dynamicSmemBytes = plan.smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)plan.splits;   // the splits of one group form one cluster
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mk, mv, dp);
 }
 
 template <typename T>
@@ -525,15 +685,14 @@ bool decode_mma_supported(int dtype, int64_t Dqk, int64_t Dv) {
 }
 
 LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev) {
-    (void)dtype;
     LaunchPlan plan{};
     const int64_t rows = (int64_t)p.group * p.Lq;
     const Shape sh = pick_shape(p.Dqk, p.Dv, rows);
     const int64_t RG = (rows + 8 * sh.nt - 1) / (8 * sh.nt);
-    const int64_t nkb = (p.Lk + 15) / 16;
+    const int64_t nkb = (p.Lk + kSK - 1) / kSK;      // slots of kSK keys
     const int64_t base = p.B * p.Hkv * RG;
     int64_t splits = (int64_t)dev.sm_count / base;   // one CTA per SM, one wave
-    const int64_t max_splits = (nkb + sh.w - 1) / sh.w;   // at least one block per consumer warp
+    const int64_t max_splits = (nkb * kNSUB + sh.w - 1) / sh.w;   // at least one sub-block per consumer warp
     if (splits > max_splits) splits = max_splits;
     if (splits > kMaxSplits - 1) splits = kMaxSplits - 1;
     if (splits < 1) splits = 1;
@@ -549,11 +708,21 @@ LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev
     plan.block = dim3((unsigned)((sh.w + 1) * 32), 1, 1);
     plan.smem_bytes = sh.smem;
     plan.splits = (int)splits;
-    plan.keys_per_split = kbps * 16;
+    plan.keys_per_split = kbps * kSK;
     plan.variant = (int)RG;
     plan.aux = sh.nt;
+    // The splits of a group merge through distributed shared memory as one cluster
+    // when every cluster of the grid fits on the device at once; else through the
+    // workspace and a per-group counter.
+    plan.cluster = 0;
+    if (splits > 1 && splits <= kMaxClusterSplits && !getenv("SDPA_DECODE_NO_CLUSTER")) {
+        const int64_t clusters = (int64_t)plan.grid.y * plan.grid.z;
+        if (active_clusters(dtype, p.Dqk, p.Dv, sh.nt, (int)splits, sh.smem) >= clusters) plan.cluster = (int)splits;
+    }
     return plan;
 }
+
+bool decode_mma_uses_cluster(const LaunchPlan& plan) { return plan.cluster > 1; }
 
 size_t decode_mma_counters(const AttnParams& p, const LaunchPlan& plan) {
     return (size_t)p.B * p.Hkv * plan.variant;
@@ -561,14 +730,16 @@ size_t decode_mma_counters(const AttnParams& p, const LaunchPlan& plan) {
 
 cudaError_t decode_mma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, int* counters,
                               cudaStream_t stream) {
-    if (plan.splits > 1 && (plan.splits >= kMaxSplits || counters == nullptr)) return cudaErrorInvalidValue;
+    if (plan.splits > 1 && !decode_mma_uses_cluster(plan) && (plan.splits >= kMaxSplits || counters == nullptr))
+        return cudaErrorInvalidValue;
+    if (decode_mma_uses_cluster(plan)) counters = nullptr;
     DecParams dp{};
     dp.p = p;
     dp.RG = plan.variant;
     dp.counters = counters;
     CUtensorMap mk, mv;
-    if (!make_tensor_map(&mk, &dp.k_ax, p.k, dtype, p.Dqk, p.Lk, p.Hkv, p.B, p.sk, 16) ||
-        !make_tensor_map(&mv, &dp.v_ax, p.v, dtype, p.Dv, p.Lk, p.Hkv, p.B, p.sv, 16))
+    if (!make_tensor_map(&mk, &dp.k_ax, p.k, dtype, p.Dqk, p.Lk, p.Hkv, p.B, p.sk, kSK) ||
+        !make_tensor_map(&mv, &dp.v_ax, p.v, dtype, p.Dv, p.Lk, p.Hkv, p.B, p.sv, kSK))
         return cudaErrorInvalidValue;
     if (dtype == 1) return launch_typed<__half>(dp, mk, mv, plan, stream);
     if (dtype == 2) return launch_typed<__nv_bfloat16>(dp, mk, mv, plan, stream);

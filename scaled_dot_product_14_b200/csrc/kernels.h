@@ -53,6 +53,7 @@ struct LaunchPlan {
     int64_t keys_per_split;
     int variant;          // kernel-specific (decode: row groups per KV head)
     int aux;              // kernel-specific (decode: 8-row n-tiles per CTA)
+    int cluster;          // decode: CTAs per thread-block cluster (0 = none)
 };
 
 struct DeviceInfo {
@@ -88,6 +89,9 @@ cudaError_t ffma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, 
 bool decode_mma_supported(int dtype, int64_t Dqk, int64_t Dv);
 LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev);
 size_t decode_mma_counters(const AttnParams& p, const LaunchPlan& plan);
+// True when the splits of a group run as one thread-block cluster and merge
+// through distributed shared memory: then no workspace or counters are needed.
+bool decode_mma_uses_cluster(const LaunchPlan& plan);
 cudaError_t decode_mma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, int* counters,
                               cudaStream_t stream);
 

@@ -176,12 +176,15 @@ struct RowSoftmax {
         }
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         l *= alpha;
-        // p = 2^(s * mul - m) on pairs (f32x2); where no key of the tile is hidden,
-        // one pair in four takes the polynomial on the FMA pipe instead of MUFU.
-        // P goes to TMEM 64 keys at a time.
+        // p = 2^(s * mul - m) on pairs (f32x2); P goes to TMEM 64 keys at a time.
+        // bf16: P is packed on the integer pipe (the conversion instruction would
+        // share the MUFU unit with the exponentials, at half their rate).  fp16
+        // keeps the conversion, and where no key of the tile is hidden one pair in
+        // four takes the FMA-pipe polynomial instead of MUFU.
+        constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
         const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(-m_use, -m_use);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // four independent sum chains
-        const bool poly = (MASK == 0 || MASK == 3) && !partial;
+        const bool poly = !kBF16 && (MASK == 0 || MASK == 3) && !partial;
 #pragma unroll
         for (int h = 0; h < kBN / 64; ++h) {
             uint32_t pr[32];
@@ -195,7 +198,7 @@ struct RowSoftmax {
                 else
                     pp = f2_pack(fast_exp2(f2_lo(x)), fast_exp2(f2_hi(x)));
                 acc[c & 3] = f2_add(acc[c & 3], pp);
-                pr[c] = pack2<T>(f2_lo(pp), f2_hi(pp));
+                pr[c] = kBF16 ? pack_bf16x2_int(f2_lo(pp), f2_hi(pp)) : pack2<T>(f2_lo(pp), f2_hi(pp));
             }
             tmem_st32(s_taddr + h * 32, pr);
         }
@@ -463,6 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // teardown: every role has drained its asynchronous work
+    __syncwarp();   // producer / MMA warps reconverge (lane 0 ran their loops) before the CTA barrier
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -690,6 +694,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
         store_o<T, DVC, C::DVP>(o_taddr, n_tiles > 0 && ok, rs.l > 0.f ? 1.f / rs.l : 0.f, og, rs.row_ok);
     }
 
+    __syncwarp();   // producer / MMA warps reconverge before the CTA barrier
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

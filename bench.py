@@ -313,7 +313,7 @@ def run_ours(args, peaks):
     if not args.no_e2e:
         result["e2e"] = e2e(S, c, t, out, stream, args, world)
     if not args.no_prefill:
-        result["prefill"] = prefill_leg(S, stream, peaks, rank, args)
+        result["prefill"] = prefill_leg(S, stream, peaks, rank, args, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if rank == 0:
@@ -322,6 +322,18 @@ def run_ours(args, peaks):
         import torch.distributed as dist
         del graph
         dist.destroy_process_group()
+
+
+def run_prefill_only(args, peaks):
+    import torch
+    import scaled_dot_product_14_b200 as S
+    from scaled_dot_product_14_b200 import build
+    if not os.path.exists(S.LIB_PATH):
+        build.build()
+    torch.cuda.set_device(0)
+    stream = torch.cuda.Stream()
+    for entry in prefill_leg(S, stream, peaks, 0, args, 0):
+        print(json.dumps(entry), flush=True)
 
 
 def e2e(S, c, t, out, stream, args, world):
@@ -360,38 +372,52 @@ def e2e(S, c, t, out, stream, args, world):
             "steps": n, "ms_per_step": round(ms / n, 4)}
 
 
-def prefill_leg(S, stream, peaks, rank, args):
+def prefill_leg(S, stream, peaks, rank, args, local=0):
+    """Each prefill workload: an untimed soak (clocks sampled meanwhile), then
+    `iters` launches each timed alone with events on the launching stream, the
+    L2 flushed (a 256 MiB write) between them."""
     import torch
     res = []
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
     for w in PREFILL_WORKLOADS:
         c, t = device_case(w, rank)
         out = torch.empty(c.B * c.Hq * c.Lq * c.Dv, dtype=t["q"].dtype, device="cuda")
         sp = stream.cuda_stream
+        clocks = ClockSampler(local) if args.prefill_soak > 0 else None
         with torch.cuda.stream(stream):
             call(S, c, t, t["k"], t["v"], out, sp)
             torch.cuda.synchronize()
-            first = time.time()
-            call(S, c, t, t["k"], t["v"], out, sp)
-            torch.cuda.synchronize()
-            one = time.time() - first
-            n = int(max(3, min(20, 2.0 / max(one, 1e-4))))
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(n):
+            if clocks:
+                clocks.start()
+                soak_end = time.time() + args.prefill_soak
+                while time.time() < soak_end:
+                    for _ in range(8):
+                        call(S, c, t, t["k"], t["v"], out, sp)
+                    stream.synchronize()
+            n = args.prefill_iters
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+            for e0, e1 in evs:
+                flush.fill_(1)
+                e0.record(stream)
                 call(S, c, t, t["k"], t["v"], out, sp)
-            e1.record(stream)
+                e1.record(stream)
         torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / n
+        clk = clocks.stop() if clocks else None
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / n
         fl = prefill_flops(w)
         tf = fl / (ms * 1e-3) / 1e12
         cnt = S.sdpa_get_counters()
-        res.append({"workload": w["name"], "ms": round(ms, 4), "tflops": round(tf, 2),
-                    "algorithmic_flops": fl, "peak_tflops": peaks["bf16_tflops"],
-                    "frac": round(tf / peaks["bf16_tflops"], 4), "bound": "tensor",
-                    "kernel": "prefill_tcgen05" if cnt["prefill_tcgen05_launches"] else "prefill_ffma",
-                    "iters": n})
+        entry = {"workload": w["name"], "ms": round(ms, 4), "tflops": round(tf, 2),
+                 "algorithmic_flops": fl, "peak_tflops": peaks["bf16_tflops"],
+                 "frac": round(tf / peaks["bf16_tflops"], 4), "bound": "tensor",
+                 "kernel": "prefill_tcgen05" if cnt["prefill_tcgen05_launches"] else "prefill_ffma",
+                 "iters": n, "l2": "flushed between timed launches"}
+        if clk:
+            entry["clocks"] = clk
+        res.append(entry)
         del t, out
         torch.cuda.empty_cache()
+    del flush
     return res
 
 
@@ -467,7 +493,15 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="run only the prefill workloads and print their lines (profiling)")
+    ap.add_argument("--prefill-iters", type=int, default=20)
+    ap.add_argument("--prefill-soak", type=float, default=1.0,
+                    help="untimed seconds per prefill workload while clocks are sampled (0: no sampling)")
     args = ap.parse_args()
+    if args.prefill_only:
+        run_prefill_only(args, load_peaks())
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -173,6 +173,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
 }
+// Per-warpgroup register budget (all 128 threads of the warpgroup execute it).
+// The increases of all warpgroups of a CTA must fit in the registers it was
+// launched with (threads x registers per thread): the launcher checks that.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+    static_assert(N >= 24 && N <= 256 && N % 8 == 0, "setmaxnreg range");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+    static_assert(N >= 24 && N <= 256 && N % 8 == 0, "setmaxnreg range");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 
 // ------------------------------------------------------------------ thread-block clusters

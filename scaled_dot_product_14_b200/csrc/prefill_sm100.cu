@@ -128,7 +128,14 @@ struct RowSoftmax {
         mask_b = reinterpret_cast<const uint8_t*>(p.mask);
     }
 
+    // `half_done(h, alpha, rescale)` runs after the P of keys [64h, 64h+64) is in
+    // TMEM (stores waited for); the caller may signal the MMA issuer there.
     __device__ __forceinline__ void tile(uint32_t s_taddr, int64_t kbase, float& alpha, bool& rescale) {
+        tile(s_taddr, kbase, alpha, rescale, [](int, float, bool) {});
+    }
+    template <typename HalfDone>
+    __device__ __forceinline__ void tile(uint32_t s_taddr, int64_t kbase, float& alpha, bool& rescale,
+                                         HalfDone&& half_done) {
         const float log2e = 1.4426950408889634f;
         uint32_t sr[kBN];
 #pragma unroll
@@ -201,10 +208,11 @@ struct RowSoftmax {
                 pr[c] = kBF16 ? pack_bf16x2_int(f2_lo(pp), f2_hi(pp)) : pack2<T>(f2_lo(pp), f2_hi(pp));
             }
             tmem_st32(s_taddr + h * 32, pr);
+            tmem_wait_st();
+            half_done(h, alpha, rescale);
         }
         const uint64_t acc2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
         l += f2_lo(acc2) + f2_hi(acc2);
-        tmem_wait_st();
     }
 };
 
@@ -479,12 +487,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------- two query tiles per CTA (ping-pong)
 // For Dv <= 128 per CTA: 256 query rows of one (batch, head) as tiles A and B
 // that share every K/V chunk.  TMEM: S_A [0,128), S_B [128,256), O_A from 256,
-// O_B from 384.  Two softmax warpgroups (warps 2-5: tile A, 6-9: tile B) take
-// turns on the tensor core: while one computes its exponentials the MMA warp
-// runs the other tile's P V and next S.  MMAs issued by one thread execute in
-// order, so S_X(j+1) may be issued right after PV_X(j), which reads P_X(j)
-// from the same TMEM columns.
-constexpr int kThreads2 = 320;   // 10 warps
+// O_B from 384.  Warpgroup 0 holds the TMA producer (warp 0) and the MMA
+// issuer (warp 1); warpgroups 1 and 2 are the softmax of tiles A and B.  The
+// two take turns on the tensor core: while one computes its exponentials the
+// MMA warp runs the other tile's P V and next S.  MMAs issued by one thread
+// execute in order, so S_X(j+1) may be issued right after PV_X(j), which reads
+// P_X(j) from the same TMEM columns.  Warpgroup 0 hands registers to the
+// softmax warpgroups (setmaxnreg), which hold a 128-wide row of S each.
+constexpr int kThreads2 = 384;     // 12 warps
+constexpr int kRegsLaunch2 = 168;  // registers per thread at launch (65536 / 384, rounded down to 8)
+constexpr int kRegsCtl2 = 88;      // warpgroup 0 after the split
+constexpr int kRegsSoftmax2 = 208; // each softmax warpgroup after the split
+static_assert(128 * kRegsCtl2 + 256 * kRegsSoftmax2 <= kThreads2 * kRegsLaunch2, "register split exceeds the pool");
 
 template <int DQK, int DVC, int NSLOT>
 struct Tc2Cfg {
@@ -492,15 +506,17 @@ struct Tc2Cfg {
     static constexpr int NBV = cdiv(DVC, 64);
     static constexpr int KSTEPS = cdiv(DQK, 16);
     static constexpr int DVP = cdiv(DVC, 16) * 16;
+    static constexpr int PER_TILE = NBQ + NBV;        // ring chunks per key tile: K(j) then V(j)
+    static constexpr int NSTAGE = NSLOT / PER_TILE;   // key tiles the ring holds
     static constexpr int Q_TILE = NBQ * kBM * 128;
     static constexpr int OFF_RING = 2 * Q_TILE;
     static constexpr int OFF_BAR = OFF_RING + NSLOT * kChunk;
-    static constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 + 2 + 2 + 1;
+    // q, K full/empty and V full/empty per stage, S full / P full / O done per tile, drain
+    static constexpr int NUM_BARS = 1 + 4 * NSTAGE + 2 + 4 + 2 + 1;
     static constexpr int SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(DVP <= 128, "two O tiles of at most 128 columns");
-    static_assert(NSLOT >= 2 * (NBQ + NBV), "ring holds K(j+1) and V(j) at once");
-    static_assert(NSLOT % (NBQ + NBV) == 0, "a tile's V chunks occupy consecutive slots");
+    static_assert(NSLOT % PER_TILE == 0 && NSTAGE >= 2, "the ring holds whole key tiles, at least two");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -519,11 +535,13 @@ __global__ void __launch_bounds__(kThreads2, 1)
     const uint32_t ring = s_base + C::OFF_RING;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* bar_q = bars;
-    uint64_t* bar_full = bars + 1;              // [NSLOT]
-    uint64_t* bar_empty = bar_full + NSLOT;     // [NSLOT]
-    uint64_t* bar_s_full = bar_empty + NSLOT;   // [2]: tile A, tile B
-    uint64_t* bar_p_full = bar_s_full + 2;      // [2]
-    uint64_t* bar_o_done = bar_p_full + 2;      // [2]
+    uint64_t* bar_kfull = bars + 1;                   // [NSTAGE]: K(j) landed
+    uint64_t* bar_kempty = bar_kfull + C::NSTAGE;     // [NSTAGE]: both tiles' S(j) done with K(j)
+    uint64_t* bar_vfull = bar_kempty + C::NSTAGE;     // [NSTAGE]: V(j) landed
+    uint64_t* bar_vempty = bar_vfull + C::NSTAGE;     // [NSTAGE]: both tiles' P V(j) done with V(j)
+    uint64_t* bar_s_full = bar_vempty + C::NSTAGE;    // [2]: tile A, tile B
+    uint64_t* bar_p_full = bar_s_full + 2;            // [2][2]: tile, half of P (keys 0-63, 64-127)
+    uint64_t* bar_o_done = bar_p_full + 4;            // [2]
     uint64_t* bar_drain = bar_o_done + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
 
@@ -542,13 +560,16 @@ __global__ void __launch_bounds__(kThreads2, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
-        for (int s = 0; s < NSLOT; ++s) {
-            mbar_init(bar_full + s, 1);
-            mbar_init(bar_empty + s, 1);
+        for (int s = 0; s < C::NSTAGE; ++s) {
+            mbar_init(bar_kfull + s, 1);
+            mbar_init(bar_kempty + s, 1);
+            mbar_init(bar_vfull + s, 1);
+            mbar_init(bar_vempty + s, 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar_s_full + s, 1);
-            mbar_init(bar_p_full + s, 128);
+            mbar_init(bar_p_full + 2 * s, 128);
+            mbar_init(bar_p_full + 2 * s + 1, 128);
             mbar_init(bar_o_done + s, 1);
         }
         mbar_init(bar_drain, 1);
@@ -562,106 +583,136 @@ __global__ void __launch_bounds__(kThreads2, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    constexpr int PER_TILE = C::NBQ + C::NBV;   // ring chunks per key tile: K(j) then V(j)
-
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer: K(j), V(j), ...
-        if (lane == 0 && n_tiles > 0) {
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            mbar_arrive_expect_tx(bar_q, 2 * C::Q_TILE);
-            for (int t2 = 0; t2 < 2; ++t2)
-                for (int c = 0; c < C::NBQ; ++c)
-                    tma_load(s_base + t2 * C::Q_TILE + c * kChunk, &tmQ, bar_q, tp.q_ax, c * 64,
-                             (int)(q0 + t2 * kBM), hq, b);
-            int seq = 0;
-            bool ok = true;
-            for (int j = 0; j < n_tiles && ok; ++j) {
-                for (int c = 0; c < PER_TILE && ok; ++c) {
-                    const int slot = seq % NSLOT;
-                    if (!(ok = wait_phase(bar_empty + slot, ((seq / NSLOT) & 1) ^ 1, kErrWaitSlot))) break;
-                    mbar_arrive_expect_tx(bar_full + slot, kChunk);
-                    if (c < C::NBQ)
-                        tma_load(ring + slot * kChunk, &tmK, bar_full + slot, tp.k_ax, c * 64, j * kBN, hkv, b);
-                    else
-                        tma_load(ring + slot * kChunk, &tmV, bar_full + slot, tp.v_ax, (c - C::NBQ) * 64, j * kBN,
-                                 hkv, b);
-                    ++seq;
-                }
-            }
-            if (!ok) {
-                wait_phase(bar_q, 0, kErrWaitTmaLoad);
-                for (int x = (seq > NSLOT ? seq - NSLOT : 0); x < seq; ++x)
-                    wait_phase(bar_full + x % NSLOT, (x / NSLOT) & 1, kErrWaitTmaLoad);
-            }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && n_tiles > 0) {
-            constexpr uint32_t idS = umma_idesc_f16(kBF16 ? 1 : 0, kBM, kBN, 0, 0);
-            bool ok = wait_phase(bar_q, 0, kErrWaitTmaLoad);
-            tc_fence_after();
-            // S_X(j) = Q_X K(j)^T; `release` frees K(j)'s chunks afterwards (tile B, the second user)
-            auto issue_s = [&](int x, int j, bool release) -> bool {
-                const uint32_t d = tmem + (uint32_t)(x * kBN);
-#pragma unroll
-                for (int c = 0; c < C::NBQ; ++c) {
-                    const int seq = j * PER_TILE + c;
-                    const int slot = seq % NSLOT;
-                    if (!wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
-                    tc_fence_after();
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        if (c * 4 + k4 >= C::KSTEPS) break;
-                        const uint64_t da = umma_desc_sw128(s_base + x * C::Q_TILE + c * kChunk + k4 * 32, 16, 1024);
-                        const uint64_t db = umma_desc_sw128(ring + slot * kChunk + k4 * 32, 16, 1024);
-                        umma_ss(d, da, db, idS, (c > 0 || k4 > 0) ? 1u : 0u);
+    // Each warpgroup sets its register budget inside its own branch, so that the
+    // compiler allots registers per role.
+    if (warp < 4) {
+        regs_dec<kRegsCtl2>();
+        if (warp == 0) {
+            // -------------------------------------------------------- TMA producer: K(j), V(j), ...
+            // K(j) and V(j) each arrive on one barrier of stage j % NSTAGE; a stage is
+            // refilled once both MMA issuers have released it.
+            if (lane == 0 && n_tiles > 0) {
+                tma_prefetch_desc(&tmQ);
+                tma_prefetch_desc(&tmK);
+                tma_prefetch_desc(&tmV);
+                mbar_arrive_expect_tx(bar_q, 2 * C::Q_TILE);
+                for (int t2 = 0; t2 < 2; ++t2)
+                    for (int c = 0; c < C::NBQ; ++c)
+                        tma_load(s_base + t2 * C::Q_TILE + c * kChunk, &tmQ, bar_q, tp.q_ax, c * 64,
+                                 (int)(q0 + t2 * kBM), hq, b);
+                bool ok = true;
+                int j = 0;
+                for (; j < n_tiles && ok; ++j) {
+                    const int st = j % C::NSTAGE;
+                    const uint32_t par = ((j / C::NSTAGE) & 1) ^ 1;
+                    const uint32_t slot0 = ring + (uint32_t)(st * C::PER_TILE) * kChunk;
+                    if (!(ok = wait_phase(bar_kempty + st, par, kErrWaitSlot))) break;
+                    mbar_arrive_expect_tx(bar_kfull + st, C::NBQ * kChunk);
+                    for (int c = 0; c < C::NBQ; ++c)
+                        tma_load(slot0 + c * kChunk, &tmK, bar_kfull + st, tp.k_ax, c * 64, j * kBN, hkv, b);
+                    if (!(ok = wait_phase(bar_vempty + st, par, kErrWaitSlot))) {
+                        // K(j) is in flight: land it before the drain below
+                        wait_phase(bar_kfull + st, (j / C::NSTAGE) & 1, kErrWaitTmaLoad);
+                        break;
                     }
-                    if (release) umma_commit(bar_empty + slot);
+                    mbar_arrive_expect_tx(bar_vfull + st, C::NBV * kChunk);
+                    for (int c = 0; c < C::NBV; ++c)
+                        tma_load(slot0 + (C::NBQ + c) * kChunk, &tmV, bar_vfull + st, tp.v_ax, c * 64, j * kBN, hkv,
+                                 b);
                 }
-                umma_commit(bar_s_full + x);
-                return true;
-            };
-            // O_X += P_X(j) V(j); `release` frees V(j)'s chunks afterwards (tile B)
-            auto issue_pv = [&](int x, int j, bool release) -> bool {
-                const uint32_t a_tmem = tmem + (uint32_t)(x * kBN);
-                const uint32_t o_col = 2 * kBN + x * 128;
-                const int seq0 = j * PER_TILE + C::NBQ;   // V(j)'s chunks are consecutive ring slots
-#pragma unroll
-                for (int c = 0; c < C::NBV; ++c)
-                    if (!wait_phase(bar_full + (seq0 + c) % NSLOT, ((seq0 + c) / NSLOT) & 1, kErrWaitTmaLoad))
-                        return false;
-                tc_fence_after();
-                constexpr uint32_t idPV = umma_idesc_f16(kBF16 ? 1 : 0, kBM, C::DVP, 0, 1);
-                const uint32_t v0 = ring + (seq0 % NSLOT) * kChunk;
-#pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {   // one MMA per 16 keys covers every value column
-                    const uint64_t db = umma_desc_sw128(v0 + kk * 2048, kChunk, 1024);
-                    umma_ts(tmem + o_col, a_tmem + kk * 8, db, idPV, (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                if (release)
-#pragma unroll
-                    for (int c = 0; c < C::NBV; ++c) umma_commit(bar_empty + (seq0 + c) % NSLOT);
-                umma_commit(bar_o_done + x);
-                return true;
-            };
-            if (ok) ok = issue_s(0, 0, false);
-            if (ok) ok = issue_s(1, 0, true);
-            for (int j = 0; j < n_tiles && ok; ++j) {
-                for (int x = 0; x < 2 && ok; ++x) {
-                    if (!(ok = wait_phase(bar_p_full + x, j & 1, kErrWaitSoftmax))) break;
-                    tc_fence_after();
-                    if (!(ok = issue_pv(x, j, x == 1))) break;
-                    if (j + 1 < n_tiles && !(ok = issue_s(x, j + 1, x == 1))) break;
+                if (!ok) {
+                    // drain: every issued load lands before the CTA's shared memory goes away
+                    wait_phase(bar_q, 0, kErrWaitTmaLoad);
+                    for (int x = (j > C::NSTAGE ? j - C::NSTAGE : 0); x < j; ++x) {
+                        wait_phase(bar_kfull + x % C::NSTAGE, (x / C::NSTAGE) & 1, kErrWaitTmaLoad);
+                        wait_phase(bar_vfull + x % C::NSTAGE, (x / C::NSTAGE) & 1, kErrWaitTmaLoad);
+                    }
                 }
             }
-            umma_commit(bar_drain);
-            wait_phase(bar_drain, 0, kErrWaitMma);
+        } else if (warp == 1) {
+            // -------------------------------------------------------- MMA issuer
+            // Per key tile j: P V and then S(j+1) of tile A, then the same of tile B,
+            // so one tile's MMAs run while the other tile's softmax computes.  MMAs
+            // issued by one thread execute in order, so S_X(j+1) may overwrite P_X(j)
+            // right after P_X(j) V(j) was issued.  The tensor pipe queues few MMAs:
+            // the readiness of V(j) and K(j+1) is polled while P(j) is still being
+            // computed, so that no barrier round trip sits between the MMAs.
+            if (lane == 0 && n_tiles > 0) {
+                constexpr uint32_t idS = umma_idesc_f16(kBF16 ? 1 : 0, kBM, kBN, 0, 0);
+                constexpr uint32_t idPV = umma_idesc_f16(kBF16 ? 1 : 0, kBM, C::DVP, 0, 1);
+                const uint64_t dsc_k = umma_desc_sw128(0, 16, 1024);       // K-major (Q, K)
+                const uint64_t dsc_v = umma_desc_sw128(0, kChunk, 1024);   // MN-major (V)
+                bool ok = wait_phase(bar_q, 0, kErrWaitTmaLoad);
+                auto issue_s = [&](int x, int j) {   // S_X(j) = Q_X K(j)^T
+                    const int st = j % C::NSTAGE;
+                    const uint32_t kb = ring + (uint32_t)(st * C::PER_TILE) * kChunk;
+                    const uint32_t qx = s_base + x * C::Q_TILE;
+#pragma unroll
+                    for (int k = 0; k < C::KSTEPS; ++k) {
+                        const uint32_t off = (uint32_t)((k >> 2) * kChunk + (k & 3) * 32);
+                        umma_ss(tmem + (uint32_t)(x * kBN), dsc_k + ((qx + off) >> 4), dsc_k + ((kb + off) >> 4), idS,
+                                k > 0 ? 1u : 0u);
+                    }
+                    if (x == 1) umma_commit(bar_kempty + st);   // tile B is K(j)'s last reader
+                    umma_commit(bar_s_full + x);
+                };
+                // O_X += P_X(j) V(j) over keys [64h, 64h+64), P_X(j) read from TMEM
+                auto issue_pv = [&](int x, int j, int h) {
+                    const int st = j % C::NSTAGE;
+                    const uint32_t v0 = ring + (uint32_t)(st * C::PER_TILE + C::NBQ) * kChunk;
+                    const uint32_t a_tmem = tmem + (uint32_t)(x * kBN);
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {   // one MMA per 16 keys covers every value column
+                        const int kk = h * 4 + k4;
+                        umma_ts(tmem + (uint32_t)(2 * kBN + x * 128), a_tmem + kk * 8, dsc_v + ((v0 + kk * 2048) >> 4),
+                                idPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    if (h == 1) {
+                        if (x == 1) umma_commit(bar_vempty + st);   // tile B is V(j)'s last reader
+                        umma_commit(bar_o_done + x);
+                    }
+                };
+                if (ok) ok = wait_phase(bar_kfull, 0, kErrWaitTmaLoad);
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(0, 0);
+                    issue_s(1, 0);
+                }
+                for (int j = 0; j < n_tiles && ok; ++j) {
+                    const int stv = j % C::NSTAGE, stk = (j + 1) % C::NSTAGE;
+                    const bool more = j + 1 < n_tiles;
+                    // non-blocking polls, answered while tile A's softmax still runs
+                    bool v_ok = mbar_try_wait(bar_vfull + stv, (j / C::NSTAGE) & 1);
+                    bool k_ok = !more || mbar_try_wait(bar_kfull + stk, ((j + 1) / C::NSTAGE) & 1);
+                    for (int x = 0; x < 2 && ok; ++x) {
+                        // the first half of P_X(j) goes into the tensor pipe while the
+                        // softmax still computes the second
+                        if (!(ok = wait_phase(bar_p_full + 2 * x, j & 1, kErrWaitSoftmax))) break;
+                        if (!v_ok && !(ok = v_ok = wait_phase(bar_vfull + stv, (j / C::NSTAGE) & 1, kErrWaitTmaLoad)))
+                            break;
+                        tc_fence_after();
+                        issue_pv(x, j, 0);
+                        if (!(ok = wait_phase(bar_p_full + 2 * x + 1, j & 1, kErrWaitSoftmax))) break;
+                        tc_fence_after();
+                        issue_pv(x, j, 1);
+                        if (more) {
+                            if (!k_ok &&
+                                !(ok = k_ok = wait_phase(bar_kfull + stk, ((j + 1) / C::NSTAGE) & 1, kErrWaitTmaLoad)))
+                                break;
+                            tc_fence_after();
+                            issue_s(x, j + 1);
+                        }
+                    }
+                }
+                // every MMA issued by this thread completes before TMEM can be freed
+                umma_commit(bar_drain);
+                wait_phase(bar_drain, 0, kErrWaitMma);
+            }
         }
     } else {
-        // ------------------------------------------------------------ softmax warpgroups (A: warps 2-5, B: 6-9)
-        const int x = (warp - 2) >> 2;         // tile of this warpgroup
+        regs_inc<kRegsSoftmax2>();
+        // ------------------------------------------------------------ softmax warpgroups (A: warps 4-7, B: 8-11)
+        const int x = (warp - 4) >> 2;         // tile of this warpgroup
         const int quad = warp & 3;             // TMEM lane quadrant
         const int r = quad * 32 + lane;
         const int64_t i = q0 + x * kBM + r;
@@ -671,21 +722,23 @@ __global__ void __launch_bounds__(kThreads2, 1)
         RowSoftmax<T, MASK> rs;
         rs.init(p, b, hq, i);
         bool ok = true;
-        for (int j = 0; j < n_tiles; ++j) {
+        for (int j = 0; j < n_tiles && ok; ++j) {
             ok = __all_sync(0xffffffffu, wait_phase(bar_s_full + x, j & 1, kErrWaitMma));
             if (!ok) break;
             tc_fence_after();
             float alpha;
             bool rescale;
-            rs.tile(s_taddr, (int64_t)j * kBN, alpha, rescale);
-            if (j > 0) {
-                ok = __all_sync(0xffffffffu, wait_phase(bar_o_done + x, (j - 1) & 1, kErrWaitMma));
-                if (!ok) break;
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale)) rescale_o<C::DVP>(o_taddr, rescale ? alpha : 1.f);
-            }
-            tc_fence_before();
-            mbar_arrive(bar_p_full + x);
+            // After each half of P: O is rescaled (before the first half, once
+            // P(j-1) V(j-1) has completed) and the MMA issuer is signalled.
+            rs.tile(s_taddr, (int64_t)j * kBN, alpha, rescale, [&](int h, float a, bool rs_needed) {
+                if (h == 0 && j > 0 && __any_sync(0xffffffffu, rs_needed)) {
+                    ok = __all_sync(0xffffffffu, wait_phase(bar_o_done + x, (j - 1) & 1, kErrWaitMma));
+                    tc_fence_after();
+                    if (ok) rescale_o<C::DVP>(o_taddr, rs_needed ? a : 1.f);
+                }
+                tc_fence_before();
+                mbar_arrive(bar_p_full + 2 * x + h);
+            });
         }
         if (ok && n_tiles > 0)
             ok = __all_sync(0xffffffffu, wait_phase(bar_o_done + x, (n_tiles - 1) & 1, kErrWaitMma));
@@ -765,14 +818,28 @@ cudaError_t launch_one(const TcParams& tp, const CUtensorMap& mq, const CUtensor
     }
 }
 
+// The pair kernel's register split (setmaxnreg) waits until the increase fits in
+// the CTA's launch registers: refuse to launch a build whose register count
+// would leave the split waiting.
+template <typename Kern>
+cudaError_t launch_split_regs(Kern kern, const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk,
+                              const CUtensorMap& mv, const LaunchPlan& plan, cudaStream_t stream) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if ((int64_t)fa.numRegs * kThreads2 < 128 * kRegsCtl2 + 256 * kRegsSoftmax2 || (int)plan.block.x != kThreads2)
+        return cudaErrorInvalidConfiguration;
+    return launch_kernel(kern, tp, mq, mk, mv, plan, stream);
+}
+
 template <typename T, int DQK, int DVC, int NSLOT>
 cudaError_t launch_two(const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const LaunchPlan& plan, cudaStream_t stream) {
     switch (tp.p.mask_kind) {
-        case 0: return launch_kernel(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 0>, tp, mq, mk, mv, plan, stream);
-        case 1: return launch_kernel(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 1>, tp, mq, mk, mv, plan, stream);
-        case 2: return launch_kernel(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 2>, tp, mq, mk, mv, plan, stream);
-        case 3: return launch_kernel(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 3>, tp, mq, mk, mv, plan, stream);
+        case 0: return launch_split_regs(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 0>, tp, mq, mk, mv, plan, stream);
+        case 1: return launch_split_regs(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 1>, tp, mq, mk, mv, plan, stream);
+        case 2: return launch_split_regs(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 2>, tp, mq, mk, mv, plan, stream);
+        case 3: return launch_split_regs(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 3>, tp, mq, mk, mv, plan, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -314,7 +314,7 @@ extern "C" int sdpa_forward(const void* q, const void* k, const void* v, void* o
         p.splits = plan.splits;
         p.keys_per_split = plan.keys_per_split;
         int* counters = nullptr;
-        if (p.splits > 1 && !(mma && decode_mma_uses_cluster(plan))) {   // cluster merges need no workspace
+        if (p.splits > 1) {
             const int64_t rows = B * Hq * Lq;
             const size_t o_bytes = (size_t)rows * p.splits * Dv * sizeof(float);
             const size_t l_bytes = (size_t)rows * p.splits * sizeof(float);
@@ -407,7 +407,9 @@ extern "C" int sdpa_last_launch_count(void) { return t_last_launches; }
 
 extern "C" int sdpa_check_device_error(void* stream_ptr, int* code_out) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_ptr);
-    const int code = take_device_error_prefill_tc(stream);
+    int code = take_device_error_prefill_tc(stream);
+    const int code_d = take_device_error_decode(stream);
+    if (code == 0 || code_d < 0) code = code_d;
     if (code_out) *code_out = code;
     if (code < 0) return SDPA_ERR_CUDA;
     return code ? SDPA_ERR_TIMEOUT : SDPA_OK;

@@ -45,14 +45,10 @@ __device__ __forceinline__ float fast_exp2(float x) {  // 2^x on the MUFU unit; 
     return y;
 }
 
-// Two non-negative floats -> bf16x2 on the integer pipe (add half an ulp of
-// bf16 to the fp32 bits, keep the upper halves with one byte permute): round
-// to nearest with ties away from zero.  Used where the packing conversion would
-// otherwise share the MUFU unit with the exponentials.
-__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
-    const uint32_t a = __float_as_uint(lo) + 0x8000u, b = __float_as_uint(hi) + 0x8000u;
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(d) : "r"(a), "r"(b));
+// max(a, b, c) in one instruction (three-input form, sm_100 and later).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
 
@@ -72,27 +68,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
-}
-
-// 2^x for both halves on the FMA and integer pipes (no MUFU).  Range reduction
-// n = round(x) through the float magic number 1.5 * 2^23, f = x - n in
-// [-1/2, 1/2], cubic p(f) ~ 2^f (least-squares fit in relative error,
-// exp2_poly_fit.py; max relative error 1.4e-4 over [-120, 8]), n added to the
-// exponent field.  Inputs are clamped at -126, so -inf gives ~1e-38, not 0:
-// callers use it only where no key is masked.
-__device__ __forceinline__ uint64_t f2_exp2_poly(uint64_t x) {
-    constexpr float kMagic = 12582912.0f;
-    constexpr uint32_t kMagicShifted = 0x4B400000u << 23;
-    const uint64_t xc = f2_pack(fmaxf(f2_lo(x), -126.f), fmaxf(f2_hi(x), -126.f));
-    const uint64_t t = f2_add(xc, f2_pack(kMagic, kMagic));
-    const uint64_t n = f2_add(t, f2_pack(-kMagic, -kMagic));
-    const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);
-    uint64_t q = f2_fma(f, f2_pack(5.502926558e-02f, 5.502926558e-02f), f2_pack(2.422569841e-01f, 2.422569841e-01f));
-    q = f2_fma(q, f, f2_pack(6.932530403e-01f, 6.932530403e-01f));
-    q = f2_fma(q, f, f2_pack(9.999513626e-01f, 9.999513626e-01f));
-    const uint32_t r0 = (uint32_t)q + ((uint32_t)t << 23) - kMagicShifted;
-    const uint32_t r1 = (uint32_t)(q >> 32) + ((uint32_t)(t >> 32) << 23) - kMagicShifted;
-    return f2_bits(r0, r1);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -170,6 +145,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
     return ok != 0;
 }
+// Non-blocking test of a phase (try_wait may suspend the thread for a while).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
 }
@@ -188,34 +171,6 @@ __device__ __forceinline__ void regs_inc() {
 }
 
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
-
-// ------------------------------------------------------------------ thread-block clusters
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-// Whole-CTA cluster barrier: release this CTA's shared-memory writes, acquire the peers'.
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
-}
-// Address of the same shared-memory location in CTA `rank` of this cluster.
-__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ float4 dsmem_ld_f32x4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
-    return v;
-}
 
 // ------------------------------------------------------------------ TMA (tensor map loads, no multicast)
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, uint64_t* bar, int c0, int c1, int c2,
@@ -236,6 +191,17 @@ __device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, u
     tma_load_4d(dst, map, bar, d0, c1, c2, c3);
 }
 
+// Whole-row box through a map built by make_tensor_map_rows.
+__device__ __forceinline__ void tma_load_rows(uint32_t dst, const CUtensorMap* map, uint64_t* bar, const MapAxes& ax,
+                                              int l, int h, int b) {
+    const int c3 = ax.h_pos ? h : 0, c4 = ax.b_pos ? b : 0;
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], "
+        "[%7];\n" ::"r"(dst),
+        "l"(map), "r"(0), "r"(l), "r"(0), "r"(c3), "r"(c4), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -249,6 +215,26 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int c
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer() - t0 > 2000000000ull) {
+            atomicCAS(&g_sdpa_device_error, 0, code);
+            return false;
+        }
+    }
+}
+
+// Bounded wait until *counter >= target (a device-scope acquire load), about
+// 2 s, then the device error flag is set and false returned.  Only for
+// counters that CTAs resident at the same time increment.
+__device__ __forceinline__ bool wait_counter_geq(const int* counter, int target, int code) {
+    auto load = [&] {
+        int v;
+        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+        return v;
+    };
+    if (load() >= target) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        if (load() >= target) return true;
         if (globaltimer() - t0 > 2000000000ull) {
             atomicCAS(&g_sdpa_device_error, 0, code);
             return false;

@@ -24,17 +24,17 @@
 //    S^T = K Q^T, so the keys fill the 16-row side of the MMA and the few query
 //    rows the 8-column side; P^T reaches the B operand of O^T += V^T P^T with
 //    one movmatrix per 8x8 block;
-//  * each CTA merges its warps, writes its split's normalised partial and
-//    log-sum-exp, and the last CTA of a (batch, KV head, row group) to finish
-//    (a counter in the workspace) merges all splits into the output and resets
-//    the counter, which the library keeps at zero between calls.
+//  * each CTA merges its warps and writes its split's normalised partial and
+//    log-sum-exp; the grid is a cooperative launch (all CTAs resident at once),
+//    so the splits of a (batch, KV head, row group) meet at a bounded barrier
+//    in the workspace and then each merges one slice of the group's output
+//    (one round trip to L2 per CTA instead of one CTA merging everything); the
+//    last CTA to leave resets the barrier, which the library keeps at zero
+//    between calls.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdlib.h>
 
-#include <map>
-#include <mutex>
-#include <tuple>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -42,23 +42,23 @@
 namespace sdpa {
 namespace {
 
-constexpr int kSK = 32;                 // keys per ring slot (one TMA box of 32 rows x 128 bytes)
-constexpr int kNSUB = kSK / 16;         // 16-key sub-blocks per slot (one consumer warp each)
-constexpr int kChunk = kSK * 128;       // one 64-element column chunk of a slot
 constexpr int kMaxSplits = 256;
-constexpr int kMaxClusterSplits = 16;   // largest (non-portable) cluster
 
 __host__ __device__ constexpr int round16(int x) { return (x + 15) / 16 * 16; }
 __host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
 
-template <int DQK, int DV, int NT, int W, int NSLOT>
+// SK keys per ring slot; a slot holds K then V, each as 64-element column chunks
+// of SK rows x 128 bytes (128-byte swizzle).
+template <int DQK, int DV, int NT, int W, int NSLOT, int SK>
 struct DecodeCfg {
+    static constexpr int NSUB = SK / 16;         // 16-key sub-blocks per slot
+    static constexpr int CHUNK = SK * 128;       // one 64-element column chunk of a slot
     static constexpr int DQKP = round16(DQK);    // MMA K extent (72 -> 80; TMA zero-fills the pad)
     static constexpr int DVP = round16(DV);
     static constexpr int NBK = cdiv(DQK, 64);    // 64-element chunks per K row block
     static constexpr int NBV = cdiv(DV, 64);
-    static constexpr int SLOT = (NBK + NBV) * kChunk;
+    static constexpr int SLOT = (NBK + NBV) * CHUNK;
     static constexpr int QS = DQKP + 8;          // Q smem row stride (elements): +16 B breaks bank conflicts
     static constexpr int ROWS = 8 * NT;          // query rows per CTA
     static constexpr int OFF_RING = align1k(ROWS * QS * 2);
@@ -69,9 +69,7 @@ struct DecodeCfg {
     static constexpr int OFF_COEF = OFF_ROWS + 2 * ROWS * 8;   // [ROWS][W + 1]: merge weights, then lse
     static constexpr int SMEM = OFF_COEF + ROWS * (W + 1) * 4 + 1024;
     static constexpr int THREADS = (W + 1) * 32;
-    static_assert((MERGE_FLOATS + ROWS * kMaxSplits) * 4 <= NSLOT * SLOT, "merge area must fit in the ring");
-    static_assert((MERGE_FLOATS + ROWS * DV + ROWS * (kMaxClusterSplits + 1)) * 4 <= NSLOT * SLOT,
-                  "cluster partials must fit in the ring");
+    static_assert(MERGE_FLOATS * 4 <= NSLOT * SLOT, "merge area must fit in the ring");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -79,7 +77,7 @@ struct DecParams {
     AttnParams p;
     MapAxes k_ax, v_ax;
     int RG;          // row groups per KV head
-    int* counters;   // [B * Hkv * RG], zero between calls
+    int* counters;   // [B * Hkv * RG][2]: arrivals, departures; zero between calls
 };
 
 // ldmatrix address of 16-byte unit `u` of row `row` in a 128-byte-swizzled chunk.
@@ -87,11 +85,12 @@ __device__ __forceinline__ uint32_t swz(uint32_t chunk, int row, int u) {
     return chunk + (uint32_t)(row * 128 + ((u ^ (row & 7)) << 4));
 }
 
-template <typename T, int DQK, int DV, int NT, int W, int NSLOT, bool CLUSTER>
+template <typename T, int DQK, int DV, int NT, int W, int NSLOT, int SK>
 __global__ void __launch_bounds__((W + 1) * 32, 1)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const DecParams dp) {
-    using C = DecodeCfg<DQK, DV, NT, W, NSLOT>;
+    using C = DecodeCfg<DQK, DV, NT, W, NSLOT, SK>;
+    constexpr int kNSUB = C::NSUB, kChunk = C::CHUNK;
     const AttnParams& p = dp.p;
     extern __shared__ unsigned char smem_dyn[];
     unsigned char* smem =
@@ -99,8 +98,6 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     T* Qs = reinterpret_cast<T*>(smem);
     const uint32_t ring = smem_u32(smem + C::OFF_RING);
     float* merge = reinterpret_cast<float*>(smem + C::OFF_RING);   // reused after the key loop
-    float* weights = merge + C::MERGE_FLOATS;                       // [ROWS][splits], last CTA only
-    float* cpart = merge + C::MERGE_FLOATS;                         // cluster path: [ROWS][DV] partial
     uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* bar_empty = bar_full + NSLOT;
     int* s_flag = reinterpret_cast<int*>(bar_empty + NSLOT);
@@ -151,9 +148,9 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         asm volatile("bar.sync 1, %0;\n" ::"n"(W * 32) : "memory");   // consumer warps only
     }
 
-    // ---- slots of this split (kSK keys each), cut at the causal horizon
-    const int64_t nsl = (p.Lk + kSK - 1) / kSK;
-    const int64_t slps = p.keys_per_split / kSK;
+    // ---- slots of this split (SK keys each), cut at the causal horizon
+    const int64_t nsl = (p.Lk + SK - 1) / SK;
+    const int64_t slps = p.keys_per_split / SK;
     const int64_t sl_begin = (int64_t)split * slps;
     int64_t sl_end = min(nsl, sl_begin + slps);
     if (p.mask_kind == 3) {
@@ -161,7 +158,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         for (int r = 0; r < C::ROWS; ++r)
             if (row0 + r < R) max_i = max(max_i, (row0 + r) % p.Lq);
         const int64_t last = max_i + p.Lk - p.Lq;   // last key any row sees
-        sl_end = min(sl_end, last < 0 ? (int64_t)0 : last / kSK + 1);
+        sl_end = min(sl_end, last < 0 ? (int64_t)0 : last / SK + 1);
     }
     const int n_slots = sl_end > sl_begin ? (int)(sl_end - sl_begin) : 0;
 
@@ -191,14 +188,23 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                 const int slot = t % NSLOT;
                 if (!(ok = wait_phase(bar_empty + slot, ((t / NSLOT) & 1) ^ 1, kErrWaitSlot))) break;
                 mbar_arrive_expect_tx(bar_full + slot, C::SLOT);
-                const int key0 = (int)((sl_begin + t) * kSK);
+                const int key0 = (int)((sl_begin + t) * SK);
                 const uint32_t base = ring + slot * C::SLOT;
+                // head dims that are multiples of 64 come as one whole-row box per
+                // tensor (one thread issuing one box per chunk cannot keep HBM busy)
+                if (DQK % 64 == 0)
+                    tma_load_rows(base, &tmK, bar_full + slot, dp.k_ax, key0, hkv, b);
+                else
 #pragma unroll
-                for (int c = 0; c < C::NBK; ++c)
-                    tma_load(base + c * kChunk, &tmK, bar_full + slot, dp.k_ax, c * 64, key0, hkv, b);
+                    for (int c = 0; c < C::NBK; ++c)
+                        tma_load(base + c * kChunk, &tmK, bar_full + slot, dp.k_ax, c * 64, key0, hkv, b);
+                if (DV % 64 == 0)
+                    tma_load_rows(base + C::NBK * kChunk, &tmV, bar_full + slot, dp.v_ax, key0, hkv, b);
+                else
 #pragma unroll
-                for (int c = 0; c < C::NBV; ++c)
-                    tma_load(base + (C::NBK + c) * kChunk, &tmV, bar_full + slot, dp.v_ax, c * 64, key0, hkv, b);
+                    for (int c = 0; c < C::NBV; ++c)
+                        tma_load(base + (C::NBK + c) * kChunk, &tmV, bar_full + slot, dp.v_ax, c * 64, key0, hkv,
+                                 b);
             }
             if (!ok)   // every issued load must land before shared memory is reused or released
                 for (int x = (t > NSLOT ? t - NSLOT : 0); x < t; ++x)
@@ -415,8 +421,6 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
             pk.x = pack2<T>(acc.x, acc.y);
             pk.y = pack2<T>(acc.z, acc.w);
             *reinterpret_cast<uint2*>(reinterpret_cast<T*>(p.out) + row_out[r] + c4 * 4) = pk;
-        } else if (CLUSTER) {
-            reinterpret_cast<float4*>(cpart)[r * (DV / 4) + c4] = acc;   // kept for the peers
         } else {
             __stcg(reinterpret_cast<float4*>(p.part_o + (row * S + split) * DV) + c4, acc);
             if (c4 == 0) __stcg(p.part_lse + row * S + split, coef[r * (W + 1) + W]);
@@ -424,139 +428,101 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     }
     if (S == 1) return;
 
-    if (CLUSTER) {
-        // ---- the S CTAs of this cluster are the S splits of one (batch, KV head, row group):
-        // each reads every peer's partial over distributed shared memory and writes a
-        // slice of the output; no global round trip, no counter.
-        cluster_sync();
-        float* wgt = cpart + C::ROWS * DV;   // [ROWS][kMaxClusterSplits]: split weights, then 1 / sum
-        for (int idx = tid; idx < C::ROWS * S; idx += C::THREADS) {
-            const int r = idx / S, s2 = idx % S;
-            wgt[r * (kMaxClusterSplits + 1) + s2] =
-                dsmem_ld_f32(dsmem_addr(coef + r * (W + 1) + W, (uint32_t)s2));   // lse of split s2
-        }
-        __syncthreads();
-        for (int r = tid; r < C::ROWS; r += C::THREADS) {
-            float* wr = wgt + r * (kMaxClusterSplits + 1);
-            float mx = -INFINITY;
-            for (int s2 = 0; s2 < S; ++s2) mx = fmaxf(mx, wr[s2]);
-            float sum = 0.f;
-            for (int s2 = 0; s2 < S; ++s2) {
-                const float ws = (mx == -INFINITY) ? 0.f : fast_exp2(wr[s2] - mx);   // -inf -> 0
-                wr[s2] = ws;
-                sum += ws;
-            }
-            wr[kMaxClusterSplits] = (sum > 0.f) ? 1.f / sum : 0.f;
-        }
-        __syncthreads();
-        const int rank = (int)cluster_ctarank();
-        for (int idx = rank * C::THREADS + tid; idx < C::ROWS * (DV / 4); idx += S * C::THREADS) {
+    // ---- the S splits of this (batch, KV head, row group) meet: arrivals are
+    // counted in the workspace (every CTA of the grid is resident: cooperative
+    // launch), then each CTA merges its slice of the group's rows x columns
+    int* counter = dp.counters + (((int64_t)b * p.Hkv + hkv) * dp.RG + rg) * 2;
+    __threadfence();   // this CTA's partials are visible before its arrival
+    __syncthreads();
+    if (tid == 0) {
+        atomicAdd(counter, 1);
+        *s_flag = wait_counter_geq(counter, S, kErrWaitSplits) ? 1 : 0;
+    }
+    __syncthreads();
+    if (*s_flag) {
+        // this split's share of the (row, 4-column) items; each thread merges
+        // its items online over the splits, 16 splits (their log-sum-exps and
+        // partials) in flight per round trip
+        const int items = C::ROWS * (DV / 4);
+        const int per = (items + S - 1) / S;
+        const int i_end = min(items, (split + 1) * per);
+        for (int idx = split * per + tid; idx < i_end; idx += C::THREADS) {
             const int r = idx / (DV / 4), c4 = idx % (DV / 4);
-            if (row_part[r] < 0) continue;
-            const float* wr = wgt + r * (kMaxClusterSplits + 1);
-            const uint32_t local = smem_u32(cpart + (r * (DV / 4) + c4) * 4);
+            const int64_t row = row_part[r];
+            if (row < 0) continue;
+            const float4* po = reinterpret_cast<const float4*>(p.part_o + row * S * DV) + c4;
+            const float* pl = p.part_lse + row * S;
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-            for (int s2 = 0; s2 < S; ++s2) {
-                uint32_t ra;
-                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local), "r"(s2));
-                const float4 v = dsmem_ld_f32x4(ra);
-                const float ws = wr[s2];
-                acc.x = fmaf(ws, v.x, acc.x);
-                acc.y = fmaf(ws, v.y, acc.y);
-                acc.z = fmaf(ws, v.z, acc.z);
-                acc.w = fmaf(ws, v.w, acc.w);
+            float mx = -INFINITY, sum = 0.f;
+            for (int s0 = 0; s0 < S; s0 += 16) {
+                float lse[16];
+                float4 v[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const bool in = s0 + u < S;
+                    lse[u] = in ? __ldcg(pl + s0 + u) : -INFINITY;
+                    v[u] = in ? __ldcg(po + (int64_t)(s0 + u) * (DV / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                float cm = mx;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) cm = fmaxf(cm, lse[u]);
+                if (cm == -INFINITY) continue;   // no key of these splits is visible
+                const float f = (mx == -INFINITY) ? 0.f : fast_exp2(mx - cm);
+                acc.x *= f;
+                acc.y *= f;
+                acc.z *= f;
+                acc.w *= f;
+                sum *= f;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const float ws = (lse[u] == -INFINITY) ? 0.f : fast_exp2(lse[u] - cm);
+                    sum += ws;
+                    acc.x = fmaf(ws, v[u].x, acc.x);
+                    acc.y = fmaf(ws, v[u].y, acc.y);
+                    acc.z = fmaf(ws, v[u].z, acc.z);
+                    acc.w = fmaf(ws, v[u].w, acc.w);
+                }
+                mx = cm;
             }
-            const float inv = wr[kMaxClusterSplits];
+            const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
             uint2 pk;
             pk.x = pack2<T>(acc.x * inv, acc.y * inv);
             pk.y = pack2<T>(acc.z * inv, acc.w * inv);
             *reinterpret_cast<uint2*>(reinterpret_cast<T*>(p.out) + row_out[r] + c4 * 4) = pk;
         }
-        cluster_sync();   // no CTA leaves while a peer may still read its shared memory
-        return;
     }
-
-    // ---- the last CTA of this (batch, KV head, row group) merges every split
-    __threadfence();
+    // the last split to leave resets the barrier for the next call on this workspace
     __syncthreads();
-    int* counter = dp.counters + ((int64_t)b * p.Hkv + hkv) * dp.RG + rg;
-    if (tid == 0) *s_flag = (atomicAdd(counter, 1) == S - 1);
-    __syncthreads();
-    if (!*s_flag) return;
-    __threadfence();
-    for (int idx = tid; idx < C::ROWS * S; idx += C::THREADS) {   // every split's lse, loaded in parallel
-        const int r = idx / S, s2 = idx % S;
-        const int64_t row = row_part[r];
-        weights[r * kMaxSplits + s2] = (row >= 0) ? __ldcg(p.part_lse + row * S + s2) : -INFINITY;
+    if (tid == 0 && atomicAdd(counter + 1, 1) == S - 1) {
+        counter[0] = 0;
+        counter[1] = 0;
     }
-    __syncthreads();
-    for (int r = tid; r < C::ROWS; r += C::THREADS) {   // lse -> weights 2^(lse - max), and 1 / sum
-        float* wr = weights + r * kMaxSplits;
-        float mx = -INFINITY;
-        for (int s2 = 0; s2 < S; ++s2) mx = fmaxf(mx, wr[s2]);
-        float sum = 0.f;
-        for (int s2 = 0; s2 < S; ++s2) {
-            const float ws = (mx == -INFINITY) ? 0.f : exp2f(wr[s2] - mx);   // -inf -> 0
-            wr[s2] = ws;
-            sum += ws;
-        }
-        wr[kMaxSplits - 1] = (sum > 0.f) ? 1.f / sum : 0.f;   // S < kMaxSplits
-    }
-    __syncthreads();
-    for (int idx = tid; idx < C::ROWS * (DV / 4); idx += C::THREADS) {
-        const int r = idx / (DV / 4), c4 = idx % (DV / 4);
-        const int64_t row = row_part[r];
-        if (row < 0) continue;
-        const float4* po = reinterpret_cast<const float4*>(p.part_o + row * S * DV) + c4;
-        const float* wr = weights + r * kMaxSplits;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s0 = 0; s0 < S; s0 += 16) {   // sixteen independent loads in flight per thread
-            float4 v[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u)
-                v[u] = (s0 + u < S) ? __ldcg(po + (int64_t)(s0 + u) * (DV / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const float ws = (s0 + u < S) ? wr[s0 + u] : 0.f;
-                acc.x = fmaf(ws, v[u].x, acc.x);
-                acc.y = fmaf(ws, v[u].y, acc.y);
-                acc.z = fmaf(ws, v[u].z, acc.z);
-                acc.w = fmaf(ws, v[u].w, acc.w);
-            }
-        }
-        const float inv = wr[kMaxSplits - 1];
-        T* og = reinterpret_cast<T*>(p.out) + row_out[r] + c4 * 4;
-        uint2 pk;
-        pk.x = pack2<T>(acc.x * inv, acc.y * inv);
-        pk.y = pack2<T>(acc.z * inv, acc.w * inv);
-        *reinterpret_cast<uint2*>(og) = pk;
-    }
-    if (tid == 0) *counter = 0;   // ready for the next call on this workspace
 }
 
 // ---------------------------------------------------------------- host side
 struct Shape {
-    int nt, w, nslot;
+    int nt, w, nslot, sk;
     size_t smem;
 };
 
-template <int DQK, int DV, int NT, int W, int NSLOT>
+template <int DQK, int DV, int NT, int W, int NSLOT, int SK>
 Shape shape_of() {
-    return Shape{NT, W, NSLOT, (size_t)DecodeCfg<DQK, DV, NT, W, NSLOT>::SMEM};
+    return Shape{NT, W, NSLOT, SK, (size_t)DecodeCfg<DQK, DV, NT, W, NSLOT, SK>::SMEM};
 }
 
-// (Dqk, Dv, W, NSLOT) per head dim; NT in {1, 2, 4} with the O^T accumulators at
-// DVP*NT/4 registers per thread (NT = 1 only at Dv = 512, NT <= 2 at Dv = 256).
+// (Dqk, Dv, W, NSLOT, SK) per head dim: about 192 KB of K/V in flight per SM
+// in slots of SK keys (32 at Dv >= 256, so that the ring keeps several slots);
+// NT in {1, 2, 4} with the O^T accumulators at DVP*NT/4 registers per
+// thread (NT = 1 only at Dv = 512, NT <= 2 at Dv = 256).
 #define SDPA_DECODE_DIMS(X) \
-    X(64, 64, 4, 24)        \
-    X(72, 72, 4, 12)        \
-    X(80, 80, 4, 12)        \
-    X(96, 96, 4, 12)        \
-    X(128, 128, 4, 12)      \
-    X(192, 128, 4, 9)       \
-    X(256, 256, 4, 6)       \
-    X(512, 512, 4, 3)
+    X(64, 64, 4, 12, 64)    \
+    X(72, 72, 4, 6, 64)     \
+    X(80, 80, 4, 6, 64)     \
+    X(96, 96, 4, 6, 64)     \
+    X(128, 128, 4, 6, 64)   \
+    X(192, 128, 4, 5, 64)   \
+    X(256, 256, 4, 6, 32)   \
+    X(512, 512, 4, 3, 32)
 
 constexpr int nt_cap(int dv) { return dv >= 512 ? 1 : (dv >= 256 ? 2 : 4); }
 constexpr int nt_fix(int want, int dv) { return want < nt_cap(dv) ? want : nt_cap(dv); }
@@ -566,97 +532,38 @@ Shape pick_shape(int64_t Dqk, int64_t Dv, int64_t rows) {
     int nt = 1;
     while (nt < need && nt < nt_cap((int)Dv)) nt *= 2;
     switch (Dqk * 1000 + Dv) {
-#define SDPA_DECODE_SHAPE(DQ, DVV, W, NS)                                \
-    case DQ * 1000 + DVV:                                                \
-        if (nt == 1) return shape_of<DQ, DVV, 1, W, NS>();               \
-        if (nt == 2) return shape_of<DQ, DVV, nt_fix(2, DVV), W, NS>();  \
-        return shape_of<DQ, DVV, nt_fix(4, DVV), W, NS>();
+#define SDPA_DECODE_SHAPE(DQ, DVV, W, NS, SK)                                \
+    case DQ * 1000 + DVV:                                                    \
+        if (nt == 1) return shape_of<DQ, DVV, 1, W, NS, SK>();               \
+        if (nt == 2) return shape_of<DQ, DVV, nt_fix(2, DVV), W, NS, SK>();  \
+        return shape_of<DQ, DVV, nt_fix(4, DVV), W, NS, SK>();
         SDPA_DECODE_DIMS(SDPA_DECODE_SHAPE)
 #undef SDPA_DECODE_SHAPE
-        default: return Shape{0, 0, 0, 0};
+        default: return Shape{0, 0, 0, 0, 0};
     }
 }
 
-// Clusters of `splits` CTAs the device can hold at once for this kernel (0 on error).
-template <typename T, int DQK, int DV, int NT, int W, int NS>
-int max_active_clusters(int splits, size_t smem) {
-    auto kern = decode_mma_kernel<T, DQK, DV, NT, W, NS, true>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
-        (splits > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)) {
-        cudaGetLastError();
-        return 0;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)splits);
-    cfg.blockDim = dim3((unsigned)((W + 1) * 32));
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)splits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
-        cudaGetLastError();
-        return 0;
-    }
-    return n;
-}
-
-int active_clusters(int dtype, int64_t Dqk, int64_t Dv, int nt, int splits, size_t smem) {
-    static std::mutex mu;
-    static std::map<std::tuple<int, int64_t, int64_t, int, int>, int> cache;
-    std::lock_guard<std::mutex> lk(mu);
-    const auto key = std::make_tuple(dtype, Dqk, Dv, nt, splits);
-    auto it = cache.find(key);
-    if (it != cache.end()) return it->second;
-    int n = 0;
-    switch (Dqk * 1000 + Dv) {
-#define SDPA_DECODE_OCC(DQ, DVV, W, NS)                                                                      \
-    case DQ * 1000 + DVV:                                                                                    \
-        if (dtype == 2)                                                                                      \
-            n = nt == 1 ? max_active_clusters<__nv_bfloat16, DQ, DVV, 1, W, NS>(splits, smem)                  \
-                : nt == 2 ? max_active_clusters<__nv_bfloat16, DQ, DVV, nt_fix(2, DVV), W, NS>(splits, smem)   \
-                          : max_active_clusters<__nv_bfloat16, DQ, DVV, nt_fix(4, DVV), W, NS>(splits, smem);  \
-        else                                                                                                 \
-            n = nt == 1 ? max_active_clusters<__half, DQ, DVV, 1, W, NS>(splits, smem)                         \
-                : nt == 2 ? max_active_clusters<__half, DQ, DVV, nt_fix(2, DVV), W, NS>(splits, smem)          \
-                          : max_active_clusters<__half, DQ, DVV, nt_fix(4, DVV), W, NS>(splits, smem);         \
-        break;
-        SDPA_DECODE_DIMS(SDPA_DECODE_OCC)
-#undef SDPA_DECODE_OCC
-        default: n = 0;
-    }
-    cache[key] = n;
-    return n;
-}
-
-template <typename T, int DQK, int DV, int NT, int W, int NS>
+// Splits > 1 meet at a barrier in the workspace, so every CTA of the grid must be
+// resident at once: a cooperative launch (which fails rather than run the grid
+// in waves).
+template <typename T, int DQK, int DV, int NT, int W, int NS, int SK>
 cudaError_t launch_one(const DecParams& dp, const CUtensorMap& mk, const CUtensorMap& mv, const LaunchPlan& plan,
                        cudaStream_t stream) {
-    const bool cluster = plan.cluster > 1;
-    auto kern = cluster ? decode_mma_kernel<T, DQK, DV, NT, W, NS, true> : decode_mma_kernel<T, DQK, DV, NT, W, NS, false>;
+    auto kern = decode_mma_kernel<T, DQK, DV, NT, W, NS, SK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
     if (e != cudaSuccess) return e;
-    if (!cluster) {
+    if (plan.splits <= 1) {
         kern<<<plan.grid, plan.block, plan.smem_bytes, stream>>>(mk, mv, dp);
         return cudaGetLastError();
     }
-    if (plan.splits > 8 && (e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
-                               cudaSuccess)
-        return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = plan.grid;
     cfg.blockDim = plan.block;
     cfg.dynamicSmemBytes = plan.smem_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)plan.splits;   // the splits of one group form one cluster
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, mk, mv, dp);
@@ -667,11 +574,11 @@ cudaError_t launch_typed(const DecParams& dp, const CUtensorMap& mk, const CUten
                          cudaStream_t s) {
     const int nt = plan.aux;
     switch (dp.p.Dqk * 1000 + dp.p.Dv) {
-#define SDPA_DECODE_LAUNCH(DQ, DVV, W, NS)                                                  \
-    case DQ * 1000 + DVV:                                                                   \
-        if (nt == 1) return launch_one<T, DQ, DVV, 1, W, NS>(dp, mk, mv, plan, s);          \
-        if (nt == 2) return launch_one<T, DQ, DVV, nt_fix(2, DVV), W, NS>(dp, mk, mv, plan, s); \
-        return launch_one<T, DQ, DVV, nt_fix(4, DVV), W, NS>(dp, mk, mv, plan, s);
+#define SDPA_DECODE_LAUNCH(DQ, DVV, W, NS, SK)                                                       \
+    case DQ * 1000 + DVV:                                                                            \
+        if (nt == 1) return launch_one<T, DQ, DVV, 1, W, NS, SK>(dp, mk, mv, plan, s);               \
+        if (nt == 2) return launch_one<T, DQ, DVV, nt_fix(2, DVV), W, NS, SK>(dp, mk, mv, plan, s);  \
+        return launch_one<T, DQ, DVV, nt_fix(4, DVV), W, NS, SK>(dp, mk, mv, plan, s);
         SDPA_DECODE_DIMS(SDPA_DECODE_LAUNCH)
 #undef SDPA_DECODE_LAUNCH
         default: return cudaErrorInvalidValue;
@@ -684,18 +591,25 @@ bool decode_mma_supported(int dtype, int64_t Dqk, int64_t Dv) {
     return (dtype == 1 || dtype == 2) && pick_shape(Dqk, Dv, 8).smem != 0;
 }
 
+// Work split.  A (batch, KV head, row group) is a group; its keys are split
+// across `splits` CTAs so that the grid fills the SMs in one wave (one CTA per
+// SM: the kernel takes most of the shared memory).
 LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev) {
+    (void)dtype;
     LaunchPlan plan{};
     const int64_t rows = (int64_t)p.group * p.Lq;
     const Shape sh = pick_shape(p.Dqk, p.Dv, rows);
     const int64_t RG = (rows + 8 * sh.nt - 1) / (8 * sh.nt);
-    const int64_t nkb = (p.Lk + kSK - 1) / kSK;      // slots of kSK keys
+    const int64_t nkb = (p.Lk + sh.sk - 1) / sh.sk;   // slots of sh.sk keys
     const int64_t base = p.B * p.Hkv * RG;
+    const int nsub = sh.sk / 16;
+    const int64_t max_splits = (nkb * nsub + sh.w - 1) / sh.w;   // at least one sub-block per consumer warp
     int64_t splits = (int64_t)dev.sm_count / base;   // one CTA per SM, one wave
-    const int64_t max_splits = (nkb * kNSUB + sh.w - 1) / sh.w;   // at least one sub-block per consumer warp
     if (splits > max_splits) splits = max_splits;
     if (splits > kMaxSplits - 1) splits = kMaxSplits - 1;
     if (splits < 1) splits = 1;
+    // debugging override; a grid that cannot be resident at once makes the
+    // cooperative launch fail with an error
     if (const char* env = getenv("SDPA_DECODE_SPLITS")) {
         const long v = strtol(env, nullptr, 10);
         if (v >= 1) splits = v < kMaxSplits - 1 ? v : kMaxSplits - 1;
@@ -708,42 +622,50 @@ LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev
     plan.block = dim3((unsigned)((sh.w + 1) * 32), 1, 1);
     plan.smem_bytes = sh.smem;
     plan.splits = (int)splits;
-    plan.keys_per_split = kbps * kSK;
+    plan.keys_per_split = kbps * sh.sk;
     plan.variant = (int)RG;
     plan.aux = sh.nt;
-    // The splits of a group merge through distributed shared memory as one cluster
-    // when every cluster of the grid fits on the device at once; else through the
-    // workspace and a per-group counter.
-    plan.cluster = 0;
-    if (splits > 1 && splits <= kMaxClusterSplits && !getenv("SDPA_DECODE_NO_CLUSTER")) {
-        const int64_t clusters = (int64_t)plan.grid.y * plan.grid.z;
-        if (active_clusters(dtype, p.Dqk, p.Dv, sh.nt, (int)splits, sh.smem) >= clusters) plan.cluster = (int)splits;
-    }
     return plan;
 }
 
-bool decode_mma_uses_cluster(const LaunchPlan& plan) { return plan.cluster > 1; }
 
 size_t decode_mma_counters(const AttnParams& p, const LaunchPlan& plan) {
-    return (size_t)p.B * p.Hkv * plan.variant;
+    return (size_t)p.B * p.Hkv * plan.variant * 2;
 }
 
 cudaError_t decode_mma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, int* counters,
                               cudaStream_t stream) {
-    if (plan.splits > 1 && !decode_mma_uses_cluster(plan) && (plan.splits >= kMaxSplits || counters == nullptr))
-        return cudaErrorInvalidValue;
-    if (decode_mma_uses_cluster(plan)) counters = nullptr;
+    if (plan.splits > 1 && (plan.splits >= kMaxSplits || counters == nullptr)) return cudaErrorInvalidValue;
     DecParams dp{};
     dp.p = p;
     dp.RG = plan.variant;
     dp.counters = counters;
+    const int sk = pick_shape(p.Dqk, p.Dv, (int64_t)p.group * p.Lq).sk;
     CUtensorMap mk, mv;
-    if (!make_tensor_map(&mk, &dp.k_ax, p.k, dtype, p.Dqk, p.Lk, p.Hkv, p.B, p.sk, kSK) ||
-        !make_tensor_map(&mv, &dp.v_ax, p.v, dtype, p.Dv, p.Lk, p.Hkv, p.B, p.sv, kSK))
-        return cudaErrorInvalidValue;
+    const bool ok_k = p.Dqk % 64 == 0
+                          ? make_tensor_map_rows(&mk, &dp.k_ax, p.k, dtype, p.Dqk, p.Lk, p.Hkv, p.B, p.sk, sk)
+                          : make_tensor_map(&mk, &dp.k_ax, p.k, dtype, p.Dqk, p.Lk, p.Hkv, p.B, p.sk, sk);
+    const bool ok_v = p.Dv % 64 == 0
+                          ? make_tensor_map_rows(&mv, &dp.v_ax, p.v, dtype, p.Dv, p.Lk, p.Hkv, p.B, p.sv, sk)
+                          : make_tensor_map(&mv, &dp.v_ax, p.v, dtype, p.Dv, p.Lk, p.Hkv, p.B, p.sv, sk);
+    if (!ok_k || !ok_v) return cudaErrorInvalidValue;
     if (dtype == 1) return launch_typed<__half>(dp, mk, mv, plan, stream);
     if (dtype == 2) return launch_typed<__nv_bfloat16>(dp, mk, mv, plan, stream);
     return cudaErrorInvalidValue;
+}
+
+int take_device_error_decode(cudaStream_t stream) {
+    int code = 0;
+    if (cudaMemcpyFromSymbolAsync(&code, g_sdpa_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, stream) !=
+        cudaSuccess)
+        return -1;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return -1;
+    if (code) {
+        const int zero = 0;
+        cudaMemcpyToSymbolAsync(g_sdpa_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream);
+        cudaStreamSynchronize(stream);
+    }
+    return code;
 }
 
 }  // namespace sdpa

@@ -20,6 +20,7 @@ enum DeviceErrorCode : int {
     kErrWaitMma = 2,         // an MMA completion never arrived
     kErrWaitSoftmax = 3,     // the softmax warps never released a buffer
     kErrWaitSlot = 4,        // a ring slot was never freed
+    kErrWaitSplits = 5,      // the splits of a decode group never all arrived
 };
 
 // Everything a kernel needs to address one attention problem.  Strides are in
@@ -53,7 +54,6 @@ struct LaunchPlan {
     int64_t keys_per_split;
     int variant;          // kernel-specific (decode: row groups per KV head)
     int aux;              // kernel-specific (decode: 8-row n-tiles per CTA)
-    int cluster;          // decode: CTAs per thread-block cluster (0 = none)
 };
 
 struct DeviceInfo {
@@ -77,6 +77,13 @@ struct MapAxes {
 bool make_tensor_map(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L, int64_t H,
                      int64_t B, const int64_t* st, int box_rows);
 
+// A 5-D map for D a multiple of 64 whose box is box_rows whole rows: dims 64
+// elements, sequence, D / 64 chunks (stride 128 bytes), head, batch; shared
+// memory gets [chunk][row][64]; 128-byte swizzle; zero fill out of bounds.
+// ax->h_pos / b_pos are 3 / 4, or 0 where the axis is pinned.  tma_map.cu.
+bool make_tensor_map_rows(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L,
+                          int64_t H, int64_t B, const int64_t* st, int box_rows);
+
 // ---- fp32 (and generic) flash kernel on CUDA cores: flash_ffma.cu
 bool ffma_supported(int dtype, int64_t Dqk, int64_t Dv);
 LaunchPlan ffma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev, bool split_keys);
@@ -89,9 +96,6 @@ cudaError_t ffma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, 
 bool decode_mma_supported(int dtype, int64_t Dqk, int64_t Dv);
 LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev);
 size_t decode_mma_counters(const AttnParams& p, const LaunchPlan& plan);
-// True when the splits of a group run as one thread-block cluster and merge
-// through distributed shared memory: then no workspace or counters are needed.
-bool decode_mma_uses_cluster(const LaunchPlan& plan);
 cudaError_t decode_mma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, int* counters,
                               cudaStream_t stream);
 
@@ -106,5 +110,6 @@ cudaError_t prefill_tc_launch(const AttnParams& p, int dtype, const LaunchPlan& 
 
 // Device error flags of each unit (read and clear; synchronous on `stream`).
 int take_device_error_prefill_tc(cudaStream_t stream);
+int take_device_error_decode(cudaStream_t stream);
 
 }  // namespace sdpa

@@ -129,7 +129,7 @@ extern "C" int sdpa_forward_noalloc(const void* q, const void* k, const void* v,
     p.splits = plan.splits;
     p.keys_per_split = plan.keys_per_split;
     int* counters = nullptr;
-    if (p.splits > 1 && !decode_mma_uses_cluster(plan)) {   // cluster merges need no scratch
+    if (p.splits > 1) {
         const int64_t rows = B * Hq * Lq;
         const size_t o_bytes = ((size_t)rows * p.splits * Dv * sizeof(float) + 255) / 256 * 256;
         const size_t l_bytes = (size_t)rows * p.splits * sizeof(float);

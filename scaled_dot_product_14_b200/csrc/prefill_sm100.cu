@@ -128,6 +128,18 @@ struct RowSoftmax {
         mask_b = reinterpret_cast<const uint8_t*>(p.mask);
     }
 
+    // 64 keys: p = 2^(x * mul - m) on pairs (MUFU), summed into acc, packed into pr.
+    __device__ __forceinline__ static void exp_half(const uint32_t* sr, uint64_t mul2, uint64_t negm2,
+                                                    uint64_t (&acc)[4], uint32_t (&pr)[32]) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+            const uint64_t x = f2_fma(f2_bits(sr[2 * c], sr[2 * c + 1]), mul2, negm2);
+            const uint64_t pp = f2_pack(fast_exp2(f2_lo(x)), fast_exp2(f2_hi(x)));
+            acc[c & 3] = f2_add(acc[c & 3], pp);
+            pr[c] = pack2<T>(f2_lo(pp), f2_hi(pp));
+        }
+    }
+
     // `half_done(h, alpha, rescale)` runs after the P of keys [64h, 64h+64) is in
     // TMEM (stores waited for); the caller may signal the MMA issuer there.
     __device__ __forceinline__ void tile(uint32_t s_taddr, int64_t kbase, float& alpha, bool& rescale) {
@@ -166,13 +178,14 @@ struct RowSoftmax {
 #pragma unroll
             for (int c = 0; c < kBN; ++c) sr[c] = (c < vis) ? sr[c] : __float_as_uint(-INFINITY);
         }
-        float mx8[8];   // eight independent chains instead of one 128-deep chain
+        float mx8[8];   // eight independent chains of three-input maxima
 #pragma unroll
         for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(sr[u]);
 #pragma unroll
-        for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
-        const float mloc = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * mul;   // scaled max
+        for (int c = 8; c < kBN; c += 2)
+            mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+        const float mloc = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                 fmaxf(mx8[6], mx8[7])) * mul;   // scaled max
         const float m_new = fmaxf(m_ref, mloc);
         alpha = 1.f;
         rescale = false;
@@ -184,29 +197,12 @@ struct RowSoftmax {
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         l *= alpha;
         // p = 2^(s * mul - m) on pairs (f32x2); P goes to TMEM 64 keys at a time.
-        // bf16: P is packed on the integer pipe (the conversion instruction would
-        // share the MUFU unit with the exponentials, at half their rate).  fp16
-        // keeps the conversion, and where no key of the tile is hidden one pair in
-        // four takes the FMA-pipe polynomial instead of MUFU.
-        constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
         const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(-m_use, -m_use);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // four independent sum chains
-        const bool poly = !kBF16 && (MASK == 0 || MASK == 3) && !partial;
 #pragma unroll
         for (int h = 0; h < kBN / 64; ++h) {
             uint32_t pr[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const int e = h * 64 + 2 * c;
-                const uint64_t x = f2_fma(f2_bits(sr[e], sr[e + 1]), mul2, negm2);
-                uint64_t pp;
-                if (poly && (c & 3) == 3)
-                    pp = f2_exp2_poly(x);
-                else
-                    pp = f2_pack(fast_exp2(f2_lo(x)), fast_exp2(f2_hi(x)));
-                acc[c & 3] = f2_add(acc[c & 3], pp);
-                pr[c] = kBF16 ? pack_bf16x2_int(f2_lo(pp), f2_hi(pp)) : pack2<T>(f2_lo(pp), f2_hi(pp));
-            }
+            exp_half(sr + h * 64, mul2, negm2, acc, pr);
             tmem_st32(s_taddr + h * 32, pr);
             tmem_wait_st();
             half_done(h, alpha, rescale);
@@ -361,13 +357,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             int seq = 0;
             bool ok = wait_phase(bar_q, 0, kErrWaitTmaLoad);
             tc_fence_after();
+            // The tensor pipe queues few MMAs, so a barrier round trip between two
+            // groups of MMAs idles it: the next chunk's barrier is polled before the
+            // current chunk's MMAs are issued, and waited on only if it was not ready.
+            auto full_ready = [&](int sq) { return mbar_test(bar_full + sq % NSLOT, (sq / NSLOT) & 1); };
             auto issue_s = [&](int j) -> bool {   // S_j = Q K_j^T into TMEM buffer j & 1
                 const uint32_t d = tmem + (uint32_t)((j & 1) * kBN);
+                bool ready = full_ready(seq);
 #pragma unroll
                 for (int c = 0; c < C::NBQ; ++c) {
                     const int slot = seq % NSLOT;
-                    if (!wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
+                    if (!ready && !wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
                     tc_fence_after();
+                    ready = (c + 1 < C::NBQ) ? full_ready(seq + 1) : true;
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
                         if (c * 4 + k4 >= C::KSTEPS) break;
@@ -381,16 +383,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(bar_s_full + (j & 1));
                 return true;
             };
-            auto issue_pv = [&](int j) -> bool {   // O += P_j V_j, P_j read from TMEM
+            // V(j) starts at ring position 2*NBQ + j*(NBQ+NBV)
+            constexpr bool kContig = v_contiguous(2 * C::NBQ, C::NBQ + C::NBV, NSLOT, C::NBV);
+            auto issue_pv = [&](int j, bool ready) -> bool {   // O += P_j V_j, P_j read from TMEM
                 const uint32_t a_tmem = tmem + (uint32_t)((j & 1) * kBN);
-                // V(j) starts at ring position 2*NBQ + j*(NBQ+NBV)
-                constexpr bool kContig = v_contiguous(2 * C::NBQ, C::NBQ + C::NBV, NSLOT, C::NBV);
                 if (kContig) {   // one MMA per 16 keys covers every value column
                     const int slot0 = seq % NSLOT;
+                    if (!ready)
 #pragma unroll
-                    for (int c = 0; c < C::NBV; ++c)
-                        if (!wait_phase(bar_full + (seq + c) % NSLOT, ((seq + c) / NSLOT) & 1, kErrWaitTmaLoad))
-                            return false;
+                        for (int c = 0; c < C::NBV; ++c)
+                            if (!wait_phase(bar_full + (seq + c) % NSLOT, ((seq + c) / NSLOT) & 1, kErrWaitTmaLoad))
+                                return false;
                     tc_fence_after();
                     constexpr uint32_t idPV = umma_idesc_f16(kBF16 ? 1 : 0, kBM, C::DVP, 0, 1);
 #pragma unroll
@@ -402,11 +405,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < C::NBV; ++c) umma_commit(bar_empty + (seq + c) % NSLOT);
                     seq += C::NBV;
                 } else {
+                    ready = ready || full_ready(seq);
 #pragma unroll
                     for (int c = 0; c < C::NBV; ++c) {
                         const int slot = seq % NSLOT;
-                        if (!wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
+                        if (!ready && !wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
                         tc_fence_after();
+                        ready = (c + 1 < C::NBV) ? full_ready(seq + 1) : true;
                         constexpr int kLastN = C::DVP - 64 * (C::NBV - 1);
                         const uint32_t idPV =
                             umma_idesc_f16(kBF16 ? 1 : 0, kBM, (c == C::NBV - 1) ? kLastN : 64, 0, 1);
@@ -425,14 +430,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             if (ok) ok = issue_s(0);
             for (int j = 0; j < n_tiles && ok; ++j) {
-                if (j + 1 < n_tiles) {
-                    // S_{j+1} reuses the TMEM buffer P_{j-1} was read from: wait for PV_{j-1}
-                    if (j >= 1 && !(ok = wait_phase(bar_o_done, (j - 1) & 1, kErrWaitMma))) break;
-                    if (!(ok = issue_s(j + 1))) break;
-                }
+                // S_{j+1} goes into the TMEM buffer that P_{j-1} was read from.  The
+                // MMAs of one thread execute in order, so it is issued right after
+                // P_{j-1} V_{j-1} without waiting for that to complete.
+                if (j + 1 < n_tiles && !(ok = issue_s(j + 1))) break;
+                // V(j)'s chunks are polled while the softmax of tile j still runs
+                bool v_ready = true;
+                if (kContig)
+#pragma unroll
+                    for (int c = 0; c < C::NBV; ++c) v_ready = full_ready(seq + c) && v_ready;
+                else
+                    v_ready = false;
                 if (!(ok = wait_phase(bar_p_full + (j & 1), (j >> 1) & 1, kErrWaitSoftmax))) break;
                 tc_fence_after();
-                if (!(ok = issue_pv(j))) break;
+                if (!(ok = issue_pv(j, v_ready))) break;
             }
             // every MMA issued by this thread completes before TMEM can be freed
             umma_commit(bar_drain);
@@ -682,8 +693,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
                     const int stv = j % C::NSTAGE, stk = (j + 1) % C::NSTAGE;
                     const bool more = j + 1 < n_tiles;
                     // non-blocking polls, answered while tile A's softmax still runs
-                    bool v_ok = mbar_try_wait(bar_vfull + stv, (j / C::NSTAGE) & 1);
-                    bool k_ok = !more || mbar_try_wait(bar_kfull + stk, ((j + 1) / C::NSTAGE) & 1);
+                    bool v_ok = mbar_test(bar_vfull + stv, (j / C::NSTAGE) & 1);
+                    bool k_ok = !more || mbar_test(bar_kfull + stk, ((j + 1) / C::NSTAGE) & 1);
                     for (int x = 0; x < 2 && ok; ++x) {
                         // the first half of P_X(j) goes into the tensor pipe while the
                         // softmax still computes the second

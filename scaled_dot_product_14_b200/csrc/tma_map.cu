@@ -81,5 +81,45 @@ bool make_tensor_map(CUtensorMap* map, MapAxes* ax, const void* base, int dtype,
     return r == CUDA_SUCCESS;
 }
 
+// A 5-D map whose box covers every 64-element chunk of a row at once (one copy
+// instead of D / 64): dim 0 = 64 elements, dim 1 = the sequence axis, dim 2 =
+// the D / 64 chunks (stride 128 bytes), dims 3 / 4 = head / batch (an extent-1
+// or zero-stride axis is pinned to coordinate 0).  D must be a multiple of 64,
+// so every chunk lies inside its row.  Shared memory receives the box chunk by
+// chunk: [chunk][row][64 elements], the layout of D / 64 separate boxes.
+bool make_tensor_map_rows(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L,
+                          int64_t H, int64_t B, const int64_t* st, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn || D % 64 != 0 || D / 64 > 256) return false;
+    const int64_t esz = 2;
+    int64_t span = D * esz;
+    const int64_t ext[3] = {L, H, B}, str[3] = {st[2] * esz, st[1] * esz, st[0] * esz};
+    for (int x = 0; x < 3; ++x)
+        if (ext[x] > 1 && str[x] > 0 && str[x] * ext[x] > span) span = str[x] * ext[x];
+    span = (span + 15) / 16 * 16;
+    cuuint64_t gdim[5] = {64, (cuuint64_t)L, (cuuint64_t)(D / 64), 1, 1};
+    cuuint64_t gstride[4] = {(cuuint64_t)(L > 1 && str[0] > 0 ? str[0] : span), 128, (cuuint64_t)span,
+                             (cuuint64_t)span};
+    ax->l_pos = 1;
+    ax->h_pos = 0;
+    ax->b_pos = 0;
+    if (H > 1 && str[1] > 0) {
+        gdim[3] = (cuuint64_t)H;
+        gstride[2] = (cuuint64_t)str[1];
+        ax->h_pos = 3;
+    }
+    if (B > 1 && str[2] > 0) {
+        gdim[4] = (cuuint64_t)B;
+        gstride[3] = (cuuint64_t)str[2];
+        ax->b_pos = 4;
+    }
+    cuuint32_t box[5] = {64, (cuuint32_t)box_rows, (cuuint32_t)(D / 64), 1, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    const CUtensorMapDataType dt =
+        dtype == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    return fn(map, dt, 5, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 }  // namespace sdpa

@@ -21,6 +21,7 @@ enum DeviceErrorCode : int {
     kErrWaitSoftmax = 3,     // the softmax warps never released a buffer
     kErrWaitSlot = 4,        // a ring slot was never freed
     kErrWaitSplits = 5,      // the splits of a decode group never all arrived
+    kErrRingLayout = 6,      // a V block would have read past the ring (never expected)
 };
 
 // Everything a kernel needs to address one attention problem.  Strides are in

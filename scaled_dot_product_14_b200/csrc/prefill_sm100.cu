@@ -54,13 +54,29 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when t
 
 __host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-// True when the NBV chunks of V(j), which start at ring position first + j * per,
-// never wrap around the NSLOT-slot ring: then one MMA with N = Dv can read all of
-// them (consecutive slots are kChunk bytes apart).
-__host__ __device__ constexpr bool v_contiguous(int first, int per, int nslot, int nbv) {
-    for (int j = 0; j < nslot; ++j)
-        if ((first + j * per) % nslot + nbv > nslot) return false;
+// The single-tile kernel's ring order: K(0), then per key tile j K(j+1) (not
+// after the last tile) and V(j).  True when, with ring positions mapped to slots
+// as (position + shift) % nslot, the NBV chunks of every V(j) occupy consecutive
+// slots for every tile count: then one MMA with N = Dv can read all of them
+// (consecutive slots are kChunk bytes apart).  The producer's position sequence
+// is replayed for up to 2 * nslot + 1 tiles, which covers every residue.
+__host__ __device__ constexpr bool v_contiguous(int nbq, int nbv, int nslot, int shift) {
+    for (int n = 1; n <= 2 * nslot + 1; ++n) {
+        int pos = nbq;   // after K(0)
+        for (int j = 0; j < n; ++j) {
+            if (j + 1 < n) pos += nbq;   // K(j+1)
+            if ((pos + shift) % nslot + nbv > nslot) return false;
+            pos += nbv;   // V(j)
+        }
+    }
     return true;
+}
+
+// The smallest slot shift that keeps every V(j) contiguous, or 0 if none does.
+__host__ __device__ constexpr int ring_shift(int nbq, int nbv, int nslot) {
+    for (int sh = 0; sh < nslot; ++sh)
+        if (v_contiguous(nbq, nbv, nslot, sh)) return sh;
+    return 0;
 }
 
 // DQK: q/k head dim; DVC: value columns this CTA produces (Dv, or Dv/2 when the
@@ -78,6 +94,8 @@ struct TcCfg {
     static constexpr int SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 1024;   // + TMEM slot + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr int O_COL = 2 * kBN;
+    static constexpr int SHIFT = ring_shift(NBQ, NBV, NSLOT);   // ring position -> slot offset
+    static constexpr bool V_CONTIG = v_contiguous(NBQ, NBV, NSLOT, SHIFT);
     static_assert(O_COL + DVP <= 512, "TMEM budget: two S buffers and O");
     static_assert(NSLOT >= 2, "ring depth");
     static_assert(SMEM <= 232448, "shared memory budget");
@@ -330,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int seq = 0;
             bool ok = true;
             auto put = [&](const CUtensorMap* map, const MapAxes& ax, int d0, int j) -> bool {
-                const int slot = seq % NSLOT;
+                const int slot = (seq + C::SHIFT) % NSLOT;
                 if (!wait_phase(bar_empty + slot, ((seq / NSLOT) & 1) ^ 1, kErrWaitSlot)) return false;
                 mbar_arrive_expect_tx(bar_full + slot, kChunk);
                 tma_load(ring + slot * kChunk, map, bar_full + slot, ax, d0, j * kBN, hkv, b);
@@ -347,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // drain: every issued load must land before the CTA's shared memory goes away
                 wait_phase(bar_q, 0, kErrWaitTmaLoad);
                 for (int x = (seq > NSLOT ? seq - NSLOT : 0); x < seq; ++x)
-                    wait_phase(bar_full + x % NSLOT, (x / NSLOT) & 1, kErrWaitTmaLoad);
+                    wait_phase(bar_full + (x + C::SHIFT) % NSLOT, (x / NSLOT) & 1, kErrWaitTmaLoad);
             }
         }
     } else if (warp == 1) {
@@ -360,13 +378,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             // The tensor pipe queues few MMAs, so a barrier round trip between two
             // groups of MMAs idles it: the next chunk's barrier is polled before the
             // current chunk's MMAs are issued, and waited on only if it was not ready.
-            auto full_ready = [&](int sq) { return mbar_test(bar_full + sq % NSLOT, (sq / NSLOT) & 1); };
+            auto full_ready = [&](int sq) { return mbar_test(bar_full + (sq + C::SHIFT) % NSLOT, (sq / NSLOT) & 1); };
             auto issue_s = [&](int j) -> bool {   // S_j = Q K_j^T into TMEM buffer j & 1
                 const uint32_t d = tmem + (uint32_t)((j & 1) * kBN);
                 bool ready = full_ready(seq);
 #pragma unroll
                 for (int c = 0; c < C::NBQ; ++c) {
-                    const int slot = seq % NSLOT;
+                    const int slot = (seq + C::SHIFT) % NSLOT;
                     if (!ready && !wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
                     tc_fence_after();
                     ready = (c + 1 < C::NBQ) ? full_ready(seq + 1) : true;
@@ -383,16 +401,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(bar_s_full + (j & 1));
                 return true;
             };
-            // V(j) starts at ring position 2*NBQ + j*(NBQ+NBV)
-            constexpr bool kContig = v_contiguous(2 * C::NBQ, C::NBQ + C::NBV, NSLOT, C::NBV);
+            constexpr bool kContig = C::V_CONTIG;
             auto issue_pv = [&](int j, bool ready) -> bool {   // O += P_j V_j, P_j read from TMEM
                 const uint32_t a_tmem = tmem + (uint32_t)((j & 1) * kBN);
                 if (kContig) {   // one MMA per 16 keys covers every value column
-                    const int slot0 = seq % NSLOT;
+                    const int slot0 = (seq + C::SHIFT) % NSLOT;
+                    if (slot0 + C::NBV > NSLOT) {   // excluded by v_contiguous; checked, never read past the ring
+                        atomicCAS(&g_sdpa_device_error, 0, kErrRingLayout);
+                        return false;
+                    }
                     if (!ready)
 #pragma unroll
                         for (int c = 0; c < C::NBV; ++c)
-                            if (!wait_phase(bar_full + (seq + c) % NSLOT, ((seq + c) / NSLOT) & 1, kErrWaitTmaLoad))
+                            if (!wait_phase(bar_full + (seq + c + C::SHIFT) % NSLOT, ((seq + c) / NSLOT) & 1, kErrWaitTmaLoad))
                                 return false;
                     tc_fence_after();
                     constexpr uint32_t idPV = umma_idesc_f16(kBF16 ? 1 : 0, kBM, C::DVP, 0, 1);
@@ -402,13 +423,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         umma_ts(tmem + C::O_COL, a_tmem + kk * 8, db, idPV, (j > 0 || kk > 0) ? 1u : 0u);
                     }
 #pragma unroll
-                    for (int c = 0; c < C::NBV; ++c) umma_commit(bar_empty + (seq + c) % NSLOT);
+                    for (int c = 0; c < C::NBV; ++c) umma_commit(bar_empty + (seq + c + C::SHIFT) % NSLOT);
                     seq += C::NBV;
                 } else {
                     ready = ready || full_ready(seq);
 #pragma unroll
                     for (int c = 0; c < C::NBV; ++c) {
-                        const int slot = seq % NSLOT;
+                        const int slot = (seq + C::SHIFT) % NSLOT;
                         if (!ready && !wait_phase(bar_full + slot, (seq / NSLOT) & 1, kErrWaitTmaLoad)) return false;
                         tc_fence_after();
                         ready = (c + 1 < C::NBV) ? full_ready(seq + 1) : true;

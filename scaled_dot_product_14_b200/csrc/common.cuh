@@ -208,13 +208,25 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
+// try_wait that may suspend the thread for up to `ns` nanoseconds; it resumes
+// as soon as the phase completes, and meanwhile takes no issue slots from the
+// warps that share its scheduler.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(ns) : "memory");
+    return ok != 0;
+}
+
 // Bounded wait on an mbarrier phase: about 2 s, then the device error flag is
-// set and false returned.  No wait in this library can spin forever.
+// set and false returned.  No wait in this library can spin forever.  The
+// thread sleeps in the barrier between checks of the time limit.
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int code) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_suspend(bar, parity, 100000u)) return true;
         if (globaltimer() - t0 > 2000000000ull) {
             atomicCAS(&g_sdpa_device_error, 0, code);
             return false;

@@ -116,15 +116,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&o)[16]) {
 }
 
 
-// ---------------------------------------------------------------- per-row softmax (shared by both kernels)
+// ---------------------------------------------------------------- per-row softmax (shared by the kernels)
 // Thread t of a softmax warpgroup owns query row t of its 128-row tile, which
-// is TMEM lane t.  For key tile j it loads that row of S, applies scale, masks
-// and the causal / sequence limits, updates the running max (log2 domain) and
-// sum, and writes P (16-bit pairs) over the first 64 columns of the same S
-// buffer.  The caller rescales O by `alpha` when `rescale` is set, after the
-// previous tile's P V has completed.
-template <typename T, int MASK>
+// is TMEM lane t.  For a key tile of NK keys it loads that row of S, applies
+// scale, masks and the causal / sequence limits, updates the running max (log2
+// domain) and sum, and writes P as 16-bit pairs to TMEM: keys [64h, 64h+64) at
+// p_taddr + h * 32 (a last block of NK % 64 keys at the end).  P may overwrite
+// the S buffer itself (p_taddr = s_taddr) or go to columns of its own.  The
+// caller rescales O by `alpha` when `rescale` is set, once the previous P V
+// has completed, before the first P block is written.
+template <typename T, int MASK, int NK = kBN>
 struct RowSoftmax {
+    static_assert(NK % 32 == 0 && NK >= 64 && NK <= kBN, "key tile of 64 to 128 keys, a multiple of 32");
+    static constexpr int NBLK = (NK + 63) / 64;   // P blocks of 64 keys (the last may hold 32)
     float m_ref, l;
     bool row_ok, pos_scale;
     float sc;
@@ -146,11 +150,12 @@ struct RowSoftmax {
         mask_b = reinterpret_cast<const uint8_t*>(p.mask);
     }
 
-    // 64 keys: p = 2^(x * mul - m) on pairs (MUFU), summed into acc, packed into pr.
-    __device__ __forceinline__ static void exp_half(const uint32_t* sr, uint64_t mul2, uint64_t negm2,
-                                                    uint64_t (&acc)[4], uint32_t (&pr)[32]) {
+    // NP pairs: p = 2^(x * mul - m) (MUFU), summed into acc, packed into pr.
+    template <int NP>
+    __device__ __forceinline__ static void exp_pairs(const uint32_t* sr, uint64_t mul2, uint64_t negm2,
+                                                     uint64_t (&acc)[4], uint32_t* pr) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < NP; ++c) {
             const uint64_t x = f2_fma(f2_bits(sr[2 * c], sr[2 * c + 1]), mul2, negm2);
             const uint64_t pp = f2_pack(fast_exp2(f2_lo(x)), fast_exp2(f2_hi(x)));
             acc[c & 3] = f2_add(acc[c & 3], pp);
@@ -158,26 +163,36 @@ struct RowSoftmax {
         }
     }
 
-    // `half_done(h, alpha, rescale)` runs after the P of keys [64h, 64h+64) is in
-    // TMEM (stores waited for); the caller may signal the MMA issuer there.
+    // Hooks: loaded() once S is in registers (its TMEM columns may then be
+    // overwritten), before_store(h, alpha, rescale) before P block h is written,
+    // after_store(h, alpha, rescale) once that store has completed.
     __device__ __forceinline__ void tile(uint32_t s_taddr, int64_t kbase, float& alpha, bool& rescale) {
-        tile(s_taddr, kbase, alpha, rescale, [](int, float, bool) {});
+        auto none = [](int, float, bool) {};
+        tile(s_taddr, s_taddr, kbase, alpha, rescale, [] {}, none, none);
     }
     template <typename HalfDone>
     __device__ __forceinline__ void tile(uint32_t s_taddr, int64_t kbase, float& alpha, bool& rescale,
                                          HalfDone&& half_done) {
+        auto none = [](int, float, bool) {};
+        tile(s_taddr, s_taddr, kbase, alpha, rescale, [] {}, none, half_done);
+    }
+    template <typename Loaded, typename Before, typename After>
+    __device__ __forceinline__ void tile(uint32_t s_taddr, uint32_t p_taddr, int64_t kbase, float& alpha,
+                                         bool& rescale, Loaded&& loaded, Before&& before_store,
+                                         After&& after_store) {
         const float log2e = 1.4426950408889634f;
-        uint32_t sr[kBN];
+        uint32_t sr[NK];
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c)
+        for (int c = 0; c < NK / 32; ++c)
             tmem_ld32(s_taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
         tmem_wait_ld();
+        loaded();
 
         // keys of this tile that the row may see: [0, vis) (sequence end, causal limit)
         int64_t lim = Lk - kbase;
         if (MASK == 3) lim = min(lim, causal_lim - kbase + 1);
-        const int vis = row_ok ? (int)max((int64_t)0, min(lim, (int64_t)kBN)) : 0;
-        const bool partial = __any_sync(0xffffffffu, vis < kBN);   // some key of the tile is hidden
+        const int vis = row_ok ? (int)max((int64_t)0, min(lim, (int64_t)NK)) : 0;
+        const bool partial = __any_sync(0xffffffffu, vis < NK);   // some key of the tile is hidden
         // values stay raw where possible and are scaled inside the exponent's FFMA
         float mul = sc;
         if (MASK == 1 || MASK == 2 || !pos_scale) {
@@ -185,7 +200,7 @@ struct RowSoftmax {
             const T* mt_row = mask_t + mrow + kbase * msm3;
             const uint8_t* mb_row = mask_b + mrow + kbase * msm3;
 #pragma unroll
-            for (int c = 0; c < kBN; ++c) {
+            for (int c = 0; c < NK; ++c) {
                 float x = __uint_as_float(sr[c]) * sc;
                 bool keep = c < vis;
                 if (MASK == 1 && keep) x += Elem<T>::to_float(mt_row[(int64_t)c * msm3]) * log2e;
@@ -194,13 +209,13 @@ struct RowSoftmax {
             }
         } else if (partial) {
 #pragma unroll
-            for (int c = 0; c < kBN; ++c) sr[c] = (c < vis) ? sr[c] : __float_as_uint(-INFINITY);
+            for (int c = 0; c < NK; ++c) sr[c] = (c < vis) ? sr[c] : __float_as_uint(-INFINITY);
         }
         float mx8[8];   // eight independent chains of three-input maxima
 #pragma unroll
         for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(sr[u]);
 #pragma unroll
-        for (int c = 8; c < kBN; c += 2)
+        for (int c = 8; c < NK; c += 2)
             mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
         const float mloc = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
                                  fmaxf(mx8[6], mx8[7])) * mul;   // scaled max
@@ -218,12 +233,19 @@ struct RowSoftmax {
         const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(-m_use, -m_use);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // four independent sum chains
 #pragma unroll
-        for (int h = 0; h < kBN / 64; ++h) {
+        for (int h = 0; h < NBLK; ++h) {
             uint32_t pr[32];
-            exp_half(sr + h * 64, mul2, negm2, acc, pr);
-            tmem_st32(s_taddr + h * 32, pr);
+            if (h * 64 + 64 <= NK) {
+                exp_pairs<32>(sr + h * 64, mul2, negm2, acc, pr);
+                before_store(h, alpha, rescale);
+                tmem_st32(p_taddr + h * 32, pr);
+            } else {   // a last block of 32 keys
+                exp_pairs<16>(sr + h * 64, mul2, negm2, acc, pr);
+                before_store(h, alpha, rescale);
+                tmem_st16(p_taddr + h * 32, pr);
+            }
             tmem_wait_st();
-            half_done(h, alpha, rescale);
+            after_store(h, alpha, rescale);
         }
         const uint64_t acc2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
         l += f2_lo(acc2) + f2_hi(acc2);
@@ -788,18 +810,281 @@ __global__ void __launch_bounds__(kThreads2, 1)
     }
 }
 
+// ---------------------------------------------------------------- two query tiles, 96-key tiles, P apart (Dv <= 96)
+// Same roles and register split as prefill_tc2_kernel, but the key tile is 96
+// keys, which leaves TMEM room for everything: S_A [0,96), S_B [96,192),
+// O_A [192,288), O_B [288,384), P_A [384,432), P_B [448,496).  P never
+// overwrites S, so S_X(j+1) is issued as soon as the softmax of tile X has read
+// S_X(j) into registers: it is ready when that softmax finishes, and the softmax
+// warpgroups, which the exponentials bind, never wait for the tensor core.  One
+// MMA issuer per tile (warps 1 and 2), so the two tiles never wait for each
+// other; K(j) and V(j) are released once both tiles' MMAs have read them.
+constexpr int kBN3 = 96;                 // keys per tile
+constexpr int kChunk3 = kBN3 * 128;      // one ring chunk: 96 rows x 64 head-dim elements (12 KB)
+
+template <int DQK, int DVC, int NSTAGE>
+struct Tc3Cfg {
+    static constexpr int NBQ = cdiv(DQK, 64);
+    static constexpr int NBV = cdiv(DVC, 64);
+    static constexpr int KSTEPS = cdiv(DQK, 16);
+    static constexpr int DVP = cdiv(DVC, 16) * 16;
+    static constexpr int PER_TILE = NBQ + NBV;        // ring chunks per key tile: K(j) then V(j)
+    static constexpr int STAGE_BYTES = PER_TILE * kChunk3;
+    static constexpr int Q_TILE = NBQ * kBM * 128;    // Q chunks hold 128 rows
+    static constexpr int OFF_RING = 2 * Q_TILE;
+    static constexpr int OFF_BAR = OFF_RING + NSTAGE * STAGE_BYTES;
+    // q; K full/empty and V full/empty per stage; S full, S read, P full, P V done per tile; drain
+    static constexpr int NUM_BARS = 1 + 4 * NSTAGE + 2 + 2 + 2 + 2 + 1;
+    static constexpr int SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t S_COL0 = 0, S_COL1 = kBN3, O_COL0 = 2 * kBN3, O_COL1 = 2 * kBN3 + 96;
+    static constexpr uint32_t P_COL0 = 384, P_COL1 = 448;   // kBN3 / 2 columns of 16-bit pairs each
+    static_assert(DVP <= 96, "O tiles of at most 96 columns");
+    static_assert(O_COL1 + 96 <= P_COL0 && P_COL1 + kBN3 / 2 <= TMEM_COLS, "TMEM layout");
+    static_assert(NSTAGE >= 2, "the ring holds at least two key tiles");
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+template <typename T, int DQK, int DVC, int NSTAGE, int MASK>
+__global__ void __launch_bounds__(kThreads2, 1)
+    prefill_tc3_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const TcParams tp) {
+    using C = Tc3Cfg<DQK, DVC, NSTAGE>;
+    constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    const AttnParams& p = tp.p;
+
+    extern __shared__ unsigned char smem_dyn[];
+    unsigned char* smem =
+        reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t ring = s_base + C::OFF_RING;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* bar_q = bars;
+    uint64_t* bar_kfull = bars + 1;                 // [NSTAGE]: K(j) landed
+    uint64_t* bar_kempty = bar_kfull + NSTAGE;      // [NSTAGE]: both tiles' S(j) done with K(j)
+    uint64_t* bar_vfull = bar_kempty + NSTAGE;      // [NSTAGE]: V(j) landed
+    uint64_t* bar_vempty = bar_vfull + NSTAGE;      // [NSTAGE]: both tiles' P V(j) done with V(j)
+    uint64_t* bar_s_full = bar_vempty + NSTAGE;     // [2]: S_X(j) computed
+    uint64_t* bar_s_read = bar_s_full + 2;          // [2]: S_X(j) read by the softmax
+    uint64_t* bar_p_full = bar_s_read + 2;          // [2]: P_X(j) written
+    uint64_t* bar_pv = bar_p_full + 2;              // [2]: P_X(j) V(j) completed
+    uint64_t* bar_drain = bar_pv + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int pair = (MASK == 3) ? (tp.q_tiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+    const int hq = blockIdx.y, b = blockIdx.z;
+    const int hkv = hq / p.group;
+    const int64_t q0 = (int64_t)pair * 2 * kBM;   // tile A rows [q0, q0+128), tile B the next 128
+
+    int64_t kv_len = p.Lk;   // keys the pair needs (tile B sees the most under causal masking)
+    if (MASK == 3) {
+        const int64_t last = q0 + 2 * kBM - 1 + p.Lk - p.Lq;
+        kv_len = last < 0 ? 0 : (last + 1 < p.Lk ? last + 1 : p.Lk);
+    }
+    const int n_tiles = (int)((kv_len + kBN3 - 1) / kBN3);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < NSTAGE; ++s) {
+            mbar_init(bar_kfull + s, 1);
+            mbar_init(bar_kempty + s, 2);   // one commit per MMA issuer
+            mbar_init(bar_vfull + s, 1);
+            mbar_init(bar_vempty + s, 2);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar_s_full + s, 1);
+            mbar_init(bar_s_read + s, 4);   // one arrival per softmax warp
+            mbar_init(bar_p_full + s, 128);
+            mbar_init(bar_pv + s, 1);
+        }
+        mbar_init(bar_drain, 2);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (warp < 4) {
+        regs_dec<kRegsCtl2>();
+        if (warp == 0) {
+            // -------------------------------------------------------- TMA producer: K(j), V(j), ...
+            if (lane == 0 && n_tiles > 0) {
+                tma_prefetch_desc(&tmQ);
+                tma_prefetch_desc(&tmK);
+                tma_prefetch_desc(&tmV);
+                mbar_arrive_expect_tx(bar_q, 2 * C::Q_TILE);
+                for (int t2 = 0; t2 < 2; ++t2)
+                    for (int c = 0; c < C::NBQ; ++c)
+                        tma_load(s_base + t2 * C::Q_TILE + c * kChunk, &tmQ, bar_q, tp.q_ax, c * 64,
+                                 (int)(q0 + t2 * kBM), hq, b);
+                bool ok = true;
+                int j = 0;
+                for (; j < n_tiles && ok; ++j) {
+                    const int st = j % NSTAGE;
+                    const uint32_t par = ((j / NSTAGE) & 1) ^ 1;
+                    const uint32_t stage = ring + (uint32_t)st * C::STAGE_BYTES;
+                    if (!(ok = wait_phase(bar_kempty + st, par, kErrWaitSlot))) break;
+                    mbar_arrive_expect_tx(bar_kfull + st, C::NBQ * kChunk3);
+                    for (int c = 0; c < C::NBQ; ++c)
+                        tma_load(stage + c * kChunk3, &tmK, bar_kfull + st, tp.k_ax, c * 64, j * kBN3, hkv, b);
+                    if (!(ok = wait_phase(bar_vempty + st, par, kErrWaitSlot))) {
+                        wait_phase(bar_kfull + st, (j / NSTAGE) & 1, kErrWaitTmaLoad);   // K(j) is in flight
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bar_vfull + st, C::NBV * kChunk3);
+                    for (int c = 0; c < C::NBV; ++c)
+                        tma_load(stage + (C::NBQ + c) * kChunk3, &tmV, bar_vfull + st, tp.v_ax, c * 64, j * kBN3,
+                                 hkv, b);
+                }
+                if (!ok) {
+                    // drain: every issued load lands before the CTA's shared memory goes away
+                    wait_phase(bar_q, 0, kErrWaitTmaLoad);
+                    for (int x = (j > NSTAGE ? j - NSTAGE : 0); x < j; ++x) {
+                        wait_phase(bar_kfull + x % NSTAGE, (x / NSTAGE) & 1, kErrWaitTmaLoad);
+                        wait_phase(bar_vfull + x % NSTAGE, (x / NSTAGE) & 1, kErrWaitTmaLoad);
+                    }
+                }
+            }
+        } else if (warp <= 2) {
+            // -------------------------------------------------------- MMA issuer of tile x
+            const int x = warp - 1;
+            if (lane == 0 && n_tiles > 0) {
+                constexpr uint32_t idS = umma_idesc_f16(kBF16 ? 1 : 0, kBM, kBN3, 0, 0);
+                constexpr uint32_t idPV = umma_idesc_f16(kBF16 ? 1 : 0, kBM, C::DVP, 0, 1);
+                const uint64_t dsc_k = umma_desc_sw128(0, 16, 1024);        // K-major (Q, K)
+                const uint64_t dsc_v = umma_desc_sw128(0, kChunk3, 1024);   // MN-major (V)
+                const uint32_t d_s = tmem + (x ? C::S_COL1 : C::S_COL0);
+                const uint32_t d_o = tmem + (x ? C::O_COL1 : C::O_COL0);
+                const uint32_t a_p = tmem + (x ? C::P_COL1 : C::P_COL0);
+                const uint32_t qx = s_base + x * C::Q_TILE;
+                auto issue_s = [&](int j) {   // S_X(j) = Q_X K(j)^T
+                    const int st = j % NSTAGE;
+                    const uint32_t kb = ring + (uint32_t)st * C::STAGE_BYTES;
+#pragma unroll
+                    for (int k = 0; k < C::KSTEPS; ++k) {
+                        const uint32_t qo = (uint32_t)((k >> 2) * kChunk + (k & 3) * 32);
+                        const uint32_t ko = (uint32_t)((k >> 2) * kChunk3 + (k & 3) * 32);
+                        umma_ss(d_s, dsc_k + ((qx + qo) >> 4), dsc_k + ((kb + ko) >> 4), idS, k > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bar_kempty + st);
+                    umma_commit(bar_s_full + x);
+                };
+                auto issue_pv = [&](int j) {   // O_X += P_X(j) V(j), one MMA per 16 keys
+                    const int st = j % NSTAGE;
+                    const uint32_t v0 = ring + (uint32_t)st * C::STAGE_BYTES + C::NBQ * kChunk3;
+#pragma unroll
+                    for (int kk = 0; kk < kBN3 / 16; ++kk)
+                        umma_ts(d_o, a_p + kk * 8, dsc_v + ((v0 + kk * 2048) >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(bar_vempty + st);
+                    umma_commit(bar_pv + x);
+                };
+                bool ok = wait_phase(bar_q, 0, kErrWaitTmaLoad) && wait_phase(bar_kfull, 0, kErrWaitTmaLoad);
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(0);
+                }
+                for (int j = 0; j < n_tiles && ok; ++j) {
+                    const int stv = j % NSTAGE, stk = (j + 1) % NSTAGE;
+                    const bool more = j + 1 < n_tiles;
+                    // non-blocking polls, answered while the softmax still runs
+                    const bool v_ok = mbar_test(bar_vfull + stv, (j / NSTAGE) & 1);
+                    const bool k_ok = !more || mbar_test(bar_kfull + stk, ((j + 1) / NSTAGE) & 1);
+                    if (more) {   // S_X(j+1) as soon as the softmax has read S_X(j)
+                        if (!(ok = wait_phase(bar_s_read + x, j & 1, kErrWaitSoftmax))) break;
+                        if (!k_ok && !(ok = wait_phase(bar_kfull + stk, ((j + 1) / NSTAGE) & 1, kErrWaitTmaLoad)))
+                            break;
+                        tc_fence_after();
+                        issue_s(j + 1);
+                    }
+                    if (!(ok = wait_phase(bar_p_full + x, j & 1, kErrWaitSoftmax))) break;
+                    if (!v_ok && !(ok = wait_phase(bar_vfull + stv, (j / NSTAGE) & 1, kErrWaitTmaLoad))) break;
+                    tc_fence_after();
+                    issue_pv(j);
+                }
+                // every MMA issued by this thread completes before TMEM can be freed
+                umma_commit(bar_drain);
+                wait_phase(bar_drain, 0, kErrWaitMma);
+            }
+        }
+    } else {
+        regs_inc<kRegsSoftmax2>();
+        // ------------------------------------------------------------ softmax warpgroups (A: warps 4-7, B: 8-11)
+        const int x = (warp - 4) >> 2;
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const int64_t i = q0 + x * kBM + r;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t s_taddr = tmem + lane_off + (x ? C::S_COL1 : C::S_COL0);
+        const uint32_t p_taddr = tmem + lane_off + (x ? C::P_COL1 : C::P_COL0);
+        const uint32_t o_taddr = tmem + lane_off + (x ? C::O_COL1 : C::O_COL0);
+        using RS = RowSoftmax<T, MASK, kBN3>;
+        RS rs;
+        rs.init(p, b, hq, i);
+        bool ok = true;
+        for (int j = 0; j < n_tiles && ok; ++j) {
+            ok = __all_sync(0xffffffffu, wait_phase(bar_s_full + x, j & 1, kErrWaitMma));
+            if (!ok) break;
+            tc_fence_after();
+            float alpha;
+            bool rescale;
+            auto loaded = [&] {   // S_X(j) is in registers: its columns may take S_X(j+1)
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_s_read + x);
+            };
+            // Before P(j) is written: P_X(j-1) V(j-1) has completed, which frees the P
+            // columns and lets O be rescaled (one wait per key tile, in order).
+            auto before_store = [&](int h, float a, bool rs_needed) {
+                if (h != 0 || j == 0) return;
+                ok = __all_sync(0xffffffffu, wait_phase(bar_pv + x, (j - 1) & 1, kErrWaitMma)) && ok;
+                tc_fence_after();
+                if (ok && __any_sync(0xffffffffu, rs_needed)) rescale_o<C::DVP>(o_taddr, rs_needed ? a : 1.f);
+            };
+            auto after_store = [&](int h, float, bool) {
+                if (h != RS::NBLK - 1) return;
+                tc_fence_before();
+                mbar_arrive(bar_p_full + x);
+            };
+            rs.tile(s_taddr, p_taddr, (int64_t)j * kBN3, alpha, rescale, loaded, before_store, after_store);
+        }
+        if (ok && n_tiles > 0)
+            ok = __all_sync(0xffffffffu, wait_phase(bar_pv + x, (uint32_t)(n_tiles - 1) & 1, kErrWaitMma));
+        tc_fence_after();
+        T* og = reinterpret_cast<T*>(p.out) + (int64_t)b * p.so[0] + (int64_t)hq * p.so[1] + i * p.so[2];
+        store_o<T, DVC, C::DVP>(o_taddr, n_tiles > 0 && ok, rs.l > 0.f ? 1.f / rs.l : 0.f, og, rs.row_ok);
+    }
+
+    __syncwarp();   // producer / MMA warps reconverge before the CTA barrier
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
 // ---------------------------------------------------------------- host side
 struct Variant {
-    int split, smem, pair;   // pair: two query tiles per CTA (ping-pong kernel)
+    int split, smem, pair;   // pair: two query tiles per CTA (the two-tile kernels)
+    int kv_rows;             // keys per K/V box (key tile)
 };
 
 template <int DQK, int DVC, int NSLOT, int SPLIT>
 Variant variant_of() {
-    return Variant{SPLIT, TcCfg<DQK, DVC, NSLOT, SPLIT>::SMEM, 0};
+    return Variant{SPLIT, TcCfg<DQK, DVC, NSLOT, SPLIT>::SMEM, 0, kBN};
 }
 template <int DQK, int DVC, int NSLOT>
 Variant variant2_of() {
-    return Variant{1, Tc2Cfg<DQK, DVC, NSLOT>::SMEM, 1};
+    return Variant{1, Tc2Cfg<DQK, DVC, NSLOT>::SMEM, 1, kBN};
+}
+template <int DQK, int DVC, int NSTAGE>
+Variant variant3_of() {
+    return Variant{1, Tc3Cfg<DQK, DVC, NSTAGE>::SMEM, 1, kBN3};
 }
 
 // One query tile per CTA: (Dqk, Dv, Dv per CTA, ring slots, CTAs per query tile).
@@ -807,13 +1092,16 @@ Variant variant2_of() {
     X(192, 128, 128, 10, 1)             \
     X(256, 256, 256, 8, 1)              \
     X(512, 512, 256, 6, 2)
-// Two query tiles per CTA: (Dqk, Dv, ring slots); slots a multiple of the chunks per key tile.
+// Two query tiles per CTA, 128-key tiles, P over S: (Dqk, Dv, ring slots), slots a
+// multiple of the chunks per key tile.
 #define SDPA_TC2_VARIANTS(X)  \
-    X(64, 64, 10)             \
-    X(72, 72, 8)              \
-    X(80, 80, 8)              \
-    X(96, 96, 8)              \
     X(128, 128, 8)
+// Two query tiles per CTA, 96-key tiles, P apart: (Dqk, Dv, key tiles in the ring).
+#define SDPA_TC3_VARIANTS(X)  \
+    X(64, 64, 4)              \
+    X(72, 72, 3)              \
+    X(80, 80, 3)              \
+    X(96, 96, 3)
 
 Variant pick(int64_t Dqk, int64_t Dv) {
     switch (Dqk * 1000 + Dv) {
@@ -825,7 +1113,11 @@ Variant pick(int64_t Dqk, int64_t Dv) {
     case DQ * 1000 + DVV: return variant2_of<DQ, DVV, NSL>();
         SDPA_TC2_VARIANTS(SDPA_TC2_PICK)
 #undef SDPA_TC2_PICK
-        default: return Variant{0, 0, 0};
+#define SDPA_TC3_PICK(DQ, DVV, NST) \
+    case DQ * 1000 + DVV: return variant3_of<DQ, DVV, NST>();
+        SDPA_TC3_VARIANTS(SDPA_TC3_PICK)
+#undef SDPA_TC3_PICK
+        default: return Variant{0, 0, 0, 0};
     }
 }
 
@@ -876,6 +1168,18 @@ cudaError_t launch_two(const TcParams& tp, const CUtensorMap& mq, const CUtensor
     }
 }
 
+template <typename T, int DQK, int DVC, int NSTAGE>
+cudaError_t launch_three(const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const LaunchPlan& plan, cudaStream_t stream) {
+    switch (tp.p.mask_kind) {
+        case 0: return launch_split_regs(prefill_tc3_kernel<T, DQK, DVC, NSTAGE, 0>, tp, mq, mk, mv, plan, stream);
+        case 1: return launch_split_regs(prefill_tc3_kernel<T, DQK, DVC, NSTAGE, 1>, tp, mq, mk, mv, plan, stream);
+        case 2: return launch_split_regs(prefill_tc3_kernel<T, DQK, DVC, NSTAGE, 2>, tp, mq, mk, mv, plan, stream);
+        case 3: return launch_split_regs(prefill_tc3_kernel<T, DQK, DVC, NSTAGE, 3>, tp, mq, mk, mv, plan, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 template <typename T>
 cudaError_t launch_typed(const TcParams& tp, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const LaunchPlan& plan, cudaStream_t s) {
@@ -888,6 +1192,10 @@ cudaError_t launch_typed(const TcParams& tp, const CUtensorMap& mq, const CUtens
     case DQ * 1000 + DVV: return launch_two<T, DQ, DVV, NSL>(tp, mq, mk, mv, plan, s);
         SDPA_TC2_VARIANTS(SDPA_TC2_LAUNCH)
 #undef SDPA_TC2_LAUNCH
+#define SDPA_TC3_LAUNCH(DQ, DVV, NST) \
+    case DQ * 1000 + DVV: return launch_three<T, DQ, DVV, NST>(tp, mq, mk, mv, plan, s);
+        SDPA_TC3_VARIANTS(SDPA_TC3_LAUNCH)
+#undef SDPA_TC3_LAUNCH
         default: return cudaErrorInvalidValue;
     }
 }
@@ -923,9 +1231,10 @@ cudaError_t prefill_tc_launch(const AttnParams& p, int dtype, const LaunchPlan& 
     tp.p = p;
     tp.q_tiles = plan.aux;
     CUtensorMap mq, mk, mv;
+    const int kv_rows = pick(p.Dqk, p.Dv).kv_rows;
     if (!make_tensor_map(&mq, &tp.q_ax, p.q, dtype, p.Dqk, p.Lq, p.Hq, p.B, p.sq, kBM) ||
-        !make_tensor_map(&mk, &tp.k_ax, p.k, dtype, p.Dqk, p.Lk, p.Hkv, p.B, p.sk, kBN) ||
-        !make_tensor_map(&mv, &tp.v_ax, p.v, dtype, p.Dv, p.Lk, p.Hkv, p.B, p.sv, kBN))
+        !make_tensor_map(&mk, &tp.k_ax, p.k, dtype, p.Dqk, p.Lk, p.Hkv, p.B, p.sk, kv_rows) ||
+        !make_tensor_map(&mv, &tp.v_ax, p.v, dtype, p.Dv, p.Lk, p.Hkv, p.B, p.sv, kv_rows))
         return cudaErrorInvalidValue;
     if (dtype == 2) return launch_typed<__nv_bfloat16>(tp, mq, mk, mv, plan, stream);
     return launch_typed<__half>(tp, mq, mk, mv, plan, stream);

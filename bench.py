@@ -291,13 +291,21 @@ def run_ours(args, peaks):
     S.sdpa_profile_enable(False)
     n_dec, ms_dec = prof["decode_mma"]
     n_cmb, ms_cmb = prof["combine"]
-    dec_us = 1e3 * ms_dec / max(n_dec, 1)
+    dec_us_isolated = 1e3 * ms_dec / max(n_dec, 1)
+    # The decode kernel is the only kernel of a step (launches_per_step == 1 on
+    # this path): its average launch duration over the timed region is the
+    # timed region's duration divided by the launches in it.
+    dec_us = 1e3 * ms_per_step / max(launches_per_step, 1)
     achieved = bytes_per_step / (dec_us * 1e-6) / 1e9
     traffic = ncu_traffic(f"decode_mma kL={args.kl}", ["decode_mma.cu", "common.cuh", "kernels.h"])
     roof = {"bound": "hbm", "kernel": "decode_mma_kernel", "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
             "traffic": traffic, "algorithmic_bytes_per_launch": bytes_per_step,
-            "kernel_us": round(dec_us, 3), "combine_us": round(1e3 * ms_cmb / max(n_cmb, 1), 3),
+            "kernel_us": round(dec_us, 3), "launches_per_step": launches_per_step,
+            "kernel_us_isolated": round(dec_us_isolated, 3),
+            "combine_us": round(1e3 * ms_cmb / max(n_cmb, 1), 3),
+            "timing": "kernel_us = timed region / launches in it (CUDA events on the launching stream); "
+                      "kernel_us_isolated = event pair around each eager launch",
             "peak_source": f"{peaks['source']} hbm_gbs (copy, burst)"}
 
     result = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": steps_run,

@@ -432,10 +432,11 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     // counted in the workspace (every CTA of the grid is resident: cooperative
     // launch), then each CTA merges its slice of the group's rows x columns
     int* counter = dp.counters + (((int64_t)b * p.Hkv + hkv) * dp.RG + rg) * 2;
-    __threadfence();   // this CTA's partials are visible before its arrival
+    // The CTA barrier orders every thread's partial stores before thread 0's
+    // arrival, whose release (cumulative) makes them visible with it.
     __syncthreads();
     if (tid == 0) {
-        atomicAdd(counter, 1);
+        asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(counter) : "memory");
         *s_flag = wait_counter_geq(counter, S, kErrWaitSplits) ? 1 : 0;
     }
     __syncthreads();

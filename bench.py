@@ -63,7 +63,12 @@ PREFILL_WORKLOADS = [
          Lk=8192, Dqk=72, Dv=72, dtype="bf16", mask="none", layout="blhd"),
     dict(name="prefill bf16 B=1 Hq=32 Hkv=4 L=4096 D=512 causal", seed=1002, B=1, Hq=32, Hkv=4, Lq=4096, Lk=4096,
          Dqk=512, Dv=512, dtype="bf16", mask="causal", layout="bhld"),
+    dict(name="prefill fp32 B=2 Hq=32 Hkv=8 L=2048 D=64 no mask (sweep row, FFMA path)", seed=1004, B=2, Hq=32,
+         Hkv=8, Lq=2048, Lk=2048, Dqk=64, Dv=64, dtype="f32", mask="none", layout="bhld"),
 ]
+
+# fp32 runs on the CUDA cores (FFMA): peak = SMs x 128 FMA lanes x 2 FLOP x max SM clock
+FFMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def decode_bytes(w):
@@ -388,6 +393,7 @@ def prefill_leg(S, stream, peaks, rank, args, local=0):
     res = []
     flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
     for w in PREFILL_WORKLOADS:
+        S.sdpa_reset_counters()   # the kernel family of this workload is read back below
         c, t = device_case(w, rank)
         out = torch.empty(c.B * c.Hq * c.Lq * c.Dv, dtype=t["q"].dtype, device="cuda")
         sp = stream.cuda_stream
@@ -415,9 +421,13 @@ def prefill_leg(S, stream, peaks, rank, args, local=0):
         fl = prefill_flops(w)
         tf = fl / (ms * 1e-3) / 1e12
         cnt = S.sdpa_get_counters()
+        fp32 = w["dtype"] == "f32"
+        peak = FFMA_TFLOPS if fp32 else peaks["bf16_tflops"]
         entry = {"workload": w["name"], "ms": round(ms, 4), "tflops": round(tf, 2),
-                 "algorithmic_flops": fl, "peak_tflops": peaks["bf16_tflops"],
-                 "frac": round(tf / peaks["bf16_tflops"], 4), "bound": "tensor",
+                 "algorithmic_flops": fl, "peak_tflops": round(peak, 1),
+                 "peak_source": "FFMA: 148 SMs x 128 lanes x 2 x 1.965 GHz (nominal)" if fp32
+                 else f"{peaks['source']} bf16_tflops (cuBLAS, burst)",
+                 "frac": round(tf / peak, 4), "bound": "alu" if fp32 else "tensor",
                  "kernel": "prefill_tcgen05" if cnt["prefill_tcgen05_launches"] else "prefill_ffma",
                  "iters": n, "l2": "flushed between timed launches"}
         if clk:

@@ -17,6 +17,7 @@
 // (running max and sum in the log2 domain, fp32).
 #include <cuda_runtime.h>
 #include <math.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -201,6 +202,321 @@ __global__ void __launch_bounds__(kThreads) flash_ffma_kernel(const AttnParams p
     }
 }
 
+// ---- register-tiled fp32 prefill ------------------------------------------
+//
+// The same online softmax, re-tiled so that the FMA units rather than shared
+// memory set the pace: a CTA owns TM = 128 group rows and streams the keys in
+// tiles of TN = 64.  Thread (ty, tx) of the 32 x 8 grid holds the scores of
+// rows 4*ty .. 4*ty+3 against keys tx, tx+8, .., tx+56 (32 accumulators) and,
+// for the P.V product, the same 4 rows against Dv/8 output columns.  Per four
+// steps along d a thread reads 4 float4 of Q and 8 float4 of K for 128 FMAs.
+//
+// Shared memory (fp32):
+//   Qt[d][row]   Q transposed once per CTA, pre-multiplied by scale*log2(e)
+//   K[key][d]    row stride DQK+4 (an odd number of 16-byte units: the eight
+//                keys tx = 0..7 a quarter-warp reads hit distinct bank groups)
+//   V[key][c]    row stride Dv
+//   Pt[key][row] P transposed; the 16-byte unit of rows 4u..4u+3 sits at unit
+//                u ^ (key & 7), so the stores of eight consecutive keys and the
+//                loads of one key are both conflict-free
+// K and V arrive by cp.async: V of tile j while its scores are computed, K of
+// tile j+1 while P.V of tile j runs.
+constexpr int kTM = 128;
+constexpr int kTN = 64;
+constexpr int kTThreads = 256;
+
+template <int DQK, int DV>
+struct TiledSmem {
+    static_assert(DQK % 8 == 0 && DV % 8 == 0, "head dims are multiples of 8");
+    static constexpr int QS = kTM;
+    static constexpr int KS = DQK + 4;
+    static_assert((KS / 4) % 2 == 1, "K row stride must be an odd number of 16-byte units");
+    static constexpr int VS = DV;
+    static constexpr int PS = kTM;
+    static constexpr int k_off = DQK * QS;
+    static constexpr int v_off = k_off + kTN * KS;
+    static constexpr int p_off = v_off + kTN * VS;
+    static constexpr size_t bytes = sizeof(float) * ((size_t)p_off + (size_t)kTN * PS);
+};
+
+// Output columns of thread tx: Dv/32 float4 groups at 32*g + 4*tx, then, for
+// the Dv % 32 left over, a float2 at 2*tx (16 columns) and/or one column at tx
+// (8 columns).  Every column belongs to exactly one of the 8 threads of a row.
+template <int DV>
+struct TiledCols {
+    static constexpr int F4 = DV / 32;
+    static constexpr bool HAS2 = (DV % 32) >= 16;
+    static constexpr bool HAS1 = (DV % 16) == 8;
+    static constexpr int NC = 4 * F4 + (HAS2 ? 2 : 0) + (HAS1 ? 1 : 0);
+    static_assert(NC * 8 == DV, "column split");
+    static constexpr int base2 = 32 * F4;
+    static constexpr int base1 = 32 * F4 + (HAS2 ? 16 : 0);
+};
+
+template <int DV>
+__device__ __forceinline__ void tiled_load_v(float (&vv)[TiledCols<DV>::NC], const float* vrow, int tx) {
+    using C = TiledCols<DV>;
+#pragma unroll
+    for (int g = 0; g < C::F4; ++g) {
+        const float4 x = *reinterpret_cast<const float4*>(vrow + 32 * g + 4 * tx);
+        vv[4 * g] = x.x; vv[4 * g + 1] = x.y; vv[4 * g + 2] = x.z; vv[4 * g + 3] = x.w;
+    }
+    if constexpr (C::HAS2) {
+        const float2 x = *reinterpret_cast<const float2*>(vrow + C::base2 + 2 * tx);
+        vv[4 * C::F4] = x.x; vv[4 * C::F4 + 1] = x.y;
+    }
+    if constexpr (C::HAS1) vv[C::NC - 1] = vrow[C::base1 + tx];
+}
+
+template <int DV, typename F>
+__device__ __forceinline__ void tiled_for_cols(int tx, F&& f) {   // f(n, column)
+    using C = TiledCols<DV>;
+#pragma unroll
+    for (int g = 0; g < C::F4; ++g)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) f(4 * g + u, 32 * g + 4 * tx + u);
+    if constexpr (C::HAS2) { f(4 * C::F4, C::base2 + 2 * tx); f(4 * C::F4 + 1, C::base2 + 2 * tx + 1); }
+    if constexpr (C::HAS1) f(C::NC - 1, C::base1 + tx);
+}
+
+// One 64-key tile of K or V (rows kt .. kt+63 of one KV head) into shared
+// memory; rows at or past `nvalid` are zero-filled (src-size 0).
+template <int D, int LD>
+__device__ __forceinline__ void tiled_issue_rows(float* dst, const float* src, int64_t row_stride, int nvalid) {
+    constexpr int CH = D / 4;   // 16-byte chunks per row
+    for (int it = threadIdx.x; it < kTN * CH; it += kTThreads) {
+        const int r = it / CH, c = it % CH;
+        const bool ok = r < nvalid;
+        const float* g = src + (ok ? (int64_t)r * row_stride : 0) + c * 4;
+        cp_async16(smem_u32(dst + r * LD + c * 4), g, ok ? 16 : 0);
+    }
+    cp_async_commit();
+}
+
+template <int DQK, int DV, int MASK, int MINB>
+__global__ void __launch_bounds__(kTThreads, MINB) flash_tiled_f32_kernel(const AttnParams p) {
+    using S = TiledSmem<DQK, DV>;
+    using C = TiledCols<DV>;
+    extern __shared__ __align__(16) float smem[];
+    float* Qt = smem;
+    float* Ks = smem + S::k_off;
+    float* Vs = smem + S::v_off;
+    float* Pt = smem + S::p_off;
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int tx = lane & 7;
+    const int ty = (tid >> 5) * 4 + (lane >> 3);
+    const int64_t G = p.group;
+    const int64_t R = G * p.Lq;
+    const int64_t row0 = (int64_t)blockIdx.x * kTM;
+    const int hkv = blockIdx.y;
+    const int b = blockIdx.z;
+
+    const float* qg = reinterpret_cast<const float*>(p.q);
+    const float* kg = reinterpret_cast<const float*>(p.k) + b * p.sk[0] + hkv * p.sk[1];
+    const float* vg = reinterpret_cast<const float*>(p.v) + b * p.sv[0] + hkv * p.sv[1];
+
+    // Key range: all keys, cut for causal at the last key any row of the CTA sees.
+    int64_t k_end = p.Lk;
+    if (MASK == 3) {
+        const int64_t last_row = min(row0 + kTM, R) - 1;
+        // rows of the CTA may span two heads; the largest query index is Lq-1
+        // unless all rows sit in one head
+        const int64_t max_i = (row0 / p.Lq == last_row / p.Lq) ? last_row % p.Lq : p.Lq - 1;
+        k_end = min(k_end, max_i + p.Lk - p.Lq + 1);
+    }
+    if (k_end > 0) tiled_issue_rows<DQK, S::KS>(Ks, kg, p.sk[2], (int)min((int64_t)kTN, k_end));
+
+    // Qt: 32 consecutive rows per warp and one 4-column chunk, so each
+    // transposed store is 32 consecutive floats.
+    for (int it = tid; it < kTM * (DQK / 4); it += kTThreads) {
+        const int rr = it % kTM, c = it / kTM;
+        const int64_t gr = row0 + rr;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (gr < R) {
+            const int64_t h = hkv * G + gr / p.Lq, i = gr % p.Lq;
+            x = __ldg(reinterpret_cast<const float4*>(qg + b * p.sq[0] + h * p.sq[1] + i * p.sq[2] + c * 4));
+        }
+        Qt[(4 * c + 0) * S::QS + rr] = x.x * p.scale_log2;
+        Qt[(4 * c + 1) * S::QS + rr] = x.y * p.scale_log2;
+        Qt[(4 * c + 2) * S::QS + rr] = x.z * p.scale_log2;
+        Qt[(4 * c + 3) * S::QS + rr] = x.w * p.scale_log2;
+    }
+
+    // This thread's four rows.
+    int64_t qi[4], moff[4];
+    bool rok[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int64_t gr = row0 + 4 * ty + i;
+        rok[i] = gr < R;
+        const int64_t h = hkv * G + (rok[i] ? gr / p.Lq : 0);
+        qi[i] = rok[i] ? gr % p.Lq : 0;
+        moff[i] = (MASK == 1 || MASK == 2) ? b * p.sm[0] + h * p.sm[1] + qi[i] * p.sm[2] : 0;
+    }
+
+    float m[4], l[4], o[4][C::NC];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        m[i] = -INFINITY;
+        l[i] = 0.f;
+#pragma unroll
+        for (int n = 0; n < C::NC; ++n) o[i][n] = 0.f;
+    }
+    const float log2e = 1.4426950408889634f;
+
+    for (int64_t kt = 0; kt < k_end; kt += kTN) {
+        const int nvalid = (int)min((int64_t)kTN, k_end - kt);
+        cp_async_wait<0>();   // K of this tile (the only group in flight)
+        __syncthreads();      // K (and Qt) visible; the previous P.V is done with V and Pt
+        tiled_issue_rows<DV, S::VS>(Vs, vg + kt * p.sv[2], p.sv[2], nvalid);
+
+        float s[4][8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) s[i][k] = 0.f;
+        const float* kb = Ks + tx * S::KS;
+        const float* qb = Qt + 4 * ty;
+#pragma unroll 1
+        for (int d = 0; d < DQK; d += 4) {
+            float4 qf[4];
+#pragma unroll
+            for (int dd = 0; dd < 4; ++dd) qf[dd] = *reinterpret_cast<const float4*>(qb + (d + dd) * S::QS);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float4 kf = *reinterpret_cast<const float4*>(kb + 8 * k * S::KS + d);
+                const float kd[4] = {kf.x, kf.y, kf.z, kf.w};
+#pragma unroll
+                for (int dd = 0; dd < 4; ++dd) {
+                    s[0][k] = fmaf(qf[dd].x, kd[dd], s[0][k]);
+                    s[1][k] = fmaf(qf[dd].y, kd[dd], s[1][k]);
+                    s[2][k] = fmaf(qf[dd].z, kd[dd], s[2][k]);
+                    s[3][k] = fmaf(qf[dd].w, kd[dd], s[3][k]);
+                }
+            }
+        }
+
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int jj = tx + 8 * k;
+                const int64_t j = kt + jj;
+                bool keep = rok[i] && jj < nvalid;
+                if (MASK == 1 && keep)
+                    s[i][k] += __ldg(reinterpret_cast<const float*>(p.mask) + moff[i] + j * p.sm[3]) * log2e;
+                if (MASK == 2 && keep)
+                    keep = __ldg(reinterpret_cast<const uint8_t*>(p.mask) + moff[i] + j * p.sm[3]) != 0;
+                if (MASK == 3) keep = keep && j <= qi[i] + p.Lk - p.Lq;
+                if (!keep) s[i][k] = -INFINITY;
+            }
+            float mx = fmaxf(fmaxf(fmaxf(s[i][0], s[i][1]), fmaxf(s[i][2], s[i][3])),
+                             fmaxf(fmaxf(s[i][4], s[i][5]), fmaxf(s[i][6], s[i][7])));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            const float m_new = fmaxf(m[i], mx);
+            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+            const float alpha = exp2f(m[i] - m_use);   // m = -inf -> 0
+            float ps = 0.f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                s[i][k] = exp2f(s[i][k] - m_use);      // -inf -> 0
+                ps += s[i][k];
+            }
+            l[i] = l[i] * alpha + ps;
+            m[i] = m_new;
+#pragma unroll
+            for (int n = 0; n < C::NC; ++n) o[i][n] *= alpha;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)   // key tx + 8k: its unit swizzle is tx
+            *reinterpret_cast<float4*>(Pt + (tx + 8 * k) * S::PS + 4 * (ty ^ tx)) =
+                make_float4(s[0][k], s[1][k], s[2][k], s[3][k]);
+
+        cp_async_wait<0>();   // V of this tile
+        __syncthreads();      // Pt and V visible; every thread is done with K
+        if (kt + kTN < k_end)
+            tiled_issue_rows<DQK, S::KS>(Ks, kg + (kt + kTN) * p.sk[2], p.sk[2], (int)min((int64_t)kTN, k_end - kt - kTN));
+
+#pragma unroll 4
+        for (int j = 0; j < kTN; ++j) {
+            const float4 pf = *reinterpret_cast<const float4*>(Pt + j * S::PS + 4 * (ty ^ (j & 7)));
+            float vv[C::NC];
+            tiled_load_v<DV>(vv, Vs + j * S::VS, tx);
+#pragma unroll
+            for (int n = 0; n < C::NC; ++n) {
+                o[0][n] = fmaf(pf.x, vv[n], o[0][n]);
+                o[1][n] = fmaf(pf.y, vv[n], o[1][n]);
+                o[2][n] = fmaf(pf.z, vv[n], o[2][n]);
+                o[3][n] = fmaf(pf.w, vv[n], o[3][n]);
+            }
+        }
+    }
+
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float li = l[i];
+        li += __shfl_xor_sync(0xffffffffu, li, 1);
+        li += __shfl_xor_sync(0xffffffffu, li, 2);
+        li += __shfl_xor_sync(0xffffffffu, li, 4);
+        if (!rok[i]) continue;
+        const float inv = (li > 0.f) ? 1.f / li : 0.f;
+        const int64_t gr = row0 + 4 * ty + i;
+        const int64_t h = hkv * G + gr / p.Lq;
+        float* og = reinterpret_cast<float*>(p.out) + b * p.so[0] + h * p.so[1] + qi[i] * p.so[2];
+        tiled_for_cols<DV>(tx, [&](int n, int c) { og[c] = o[i][n] * inv; });
+    }
+}
+
+template <int DQK, int DV, int MASK>
+cudaError_t launch_tiled_mask(const AttnParams& p, const LaunchPlan& plan, cudaStream_t stream) {
+    constexpr int MINB = TiledSmem<DQK, DV>::bytes <= 110 * 1024 ? 2 : 1;
+    auto kern = flash_tiled_f32_kernel<DQK, DV, MASK, MINB>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
+    if (e != cudaSuccess) return e;
+    kern<<<plan.grid, plan.block, plan.smem_bytes, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <int DQK, int DV>
+cudaError_t launch_tiled(const AttnParams& p, const LaunchPlan& plan, cudaStream_t s) {
+    switch (p.mask_kind) {
+        case 0: return launch_tiled_mask<DQK, DV, 0>(p, plan, s);
+        case 1: return launch_tiled_mask<DQK, DV, 1>(p, plan, s);
+        case 2: return launch_tiled_mask<DQK, DV, 2>(p, plan, s);
+        case 3: return launch_tiled_mask<DQK, DV, 3>(p, plan, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// Head dims of the tiled kernel (Dv <= 128 keeps the accumulators in registers).
+size_t tiled_smem_for(int64_t Dqk, int64_t Dv) {
+    switch (Dqk * 1000 + Dv) {
+        case 64064: return TiledSmem<64, 64>::bytes;
+        case 72072: return TiledSmem<72, 72>::bytes;
+        case 80080: return TiledSmem<80, 80>::bytes;
+        case 96096: return TiledSmem<96, 96>::bytes;
+        case 128128: return TiledSmem<128, 128>::bytes;
+        case 192128: return TiledSmem<192, 128>::bytes;
+        default: return 0;
+    }
+}
+
+cudaError_t launch_tiled_dims(const AttnParams& p, const LaunchPlan& plan, cudaStream_t s) {
+    switch (p.Dqk * 1000 + p.Dv) {
+        case 64064: return launch_tiled<64, 64>(p, plan, s);
+        case 72072: return launch_tiled<72, 72>(p, plan, s);
+        case 80080: return launch_tiled<80, 80>(p, plan, s);
+        case 96096: return launch_tiled<96, 96>(p, plan, s);
+        case 128128: return launch_tiled<128, 128>(p, plan, s);
+        case 192128: return launch_tiled<192, 128>(p, plan, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 template <typename T, int DQK, int DV>
 cudaError_t launch_one(const AttnParams& p, const LaunchPlan& plan, cudaStream_t stream) {
     auto kern = flash_ffma_kernel<T, DQK, DV>;
@@ -246,8 +562,19 @@ bool ffma_supported(int dtype, int64_t Dqk, int64_t Dv) {
 }
 
 LaunchPlan ffma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev, bool split_keys) {
-    (void)dtype;
     LaunchPlan plan{};
+    const size_t tiled = tiled_smem_for(p.Dqk, p.Dv);
+    if (!split_keys && dtype == 0 && tiled != 0 && !getenv("SDPA_FFMA_UNTILED")) {
+        // fp32 prefill: the register-tiled kernel, one CTA per 128 group rows
+        const int64_t R = (int64_t)p.group * p.Lq;
+        plan.grid = dim3((unsigned)((R + kTM - 1) / kTM), (unsigned)p.Hkv, (unsigned)p.B);
+        plan.block = dim3(kTThreads);
+        plan.smem_bytes = tiled;
+        plan.splits = 1;
+        plan.keys_per_split = p.Lk;
+        plan.variant = 1;
+        return plan;
+    }
     const int64_t R = (int64_t)p.group * p.Lq;
     const int64_t row_tiles = (R + kRT - 1) / kRT;
     int splits = 1;
@@ -278,6 +605,7 @@ LaunchPlan ffma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev, bool
 }
 
 cudaError_t ffma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, cudaStream_t stream) {
+    if (plan.variant == 1) return dtype == 0 ? launch_tiled_dims(p, plan, stream) : cudaErrorInvalidValue;
     switch (dtype) {
         case 0: return launch_typed<float>(p, plan, stream);
         case 1: return launch_typed<__half>(p, plan, stream);

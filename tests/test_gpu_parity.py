@@ -272,6 +272,19 @@ def test_layouts_agree_on_gpu():
     assert np.abs(ga - gb).max() <= 1e-6
 
 
+@pytest.mark.parametrize("D,Dv", [(64, 64), (72, 72), (80, 80), (96, 96), (128, 128), (192, 128)])
+@pytest.mark.parametrize("mask", MASKS)
+def test_fp32_tiled_prefill_tiles(D, Dv, mask):
+    """fp32 prefill on the register-tiled kernel (128 group rows per CTA, 64-key
+    tiles): Lq=100 with 4 query heads per KV head puts rows of two heads in one
+    row tile, and Lk=200 leaves a ragged last key tile."""
+    c = I.make_case(1900 + D, 2, 8, 2, 100, 200, D, Dv, dtype=I.F32, mask=mask, layout="blhd", p_keep=0.7)
+    before = S.sdpa_get_counters()
+    run_and_check(c, label=f"fp32 tiled D={D} {mask}")
+    after = S.sdpa_get_counters()
+    assert after["prefill_ffma_launches"] == before["prefill_ffma_launches"] + 1
+
+
 def test_fp32_keeps_fp32_precision():
     """mlxcel issue #1065: fp32 error near 2^-10 = 9.77e-4 would mean reduced
     internal precision; the fp32 path must stay far below it on both paths."""

@@ -112,13 +112,21 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     const int64_t G = p.group, R = G * p.Lq;
     const int64_t row0 = (int64_t)rg * C::ROWS;
 
+    // Let the next kernel of the stream start its own launch now; nothing of
+    // this grid is read by it before its griddepcontrol.wait.
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     if (tid == 0) {
         for (int s = 0; s < NSLOT; ++s) {
             mbar_init(bar_full + s, 1);
             mbar_init(bar_empty + s, kNSUB);   // each 16-key sub-block's consumer arrives once
         }
         fence_barrier_init();
+        tma_prefetch_desc(&tmK);   // kernel parameters: safe before the wait below
+        tma_prefetch_desc(&tmV);
     }
+    // Inputs and the split counters may come from the previous kernel of the
+    // stream: wait for it to complete before the first global access.
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
     __syncthreads();   // barriers initialised; the producer starts streaming K/V right away
     if (warp > 0) {
         // ---- Q rows of this CTA (zero rows past the group and zero pad columns), consumer warps only
@@ -180,8 +188,6 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && n_slots > 0) {
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
             int t = 0;
             bool ok = true;
             for (; t < n_slots; ++t) {
@@ -553,20 +559,26 @@ cudaError_t launch_one(const DecParams& dp, const CUtensorMap& mk, const CUtenso
     auto kern = decode_mma_kernel<T, DQK, DV, NT, W, NS, SK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
     if (e != cudaSuccess) return e;
-    if (plan.splits <= 1) {
-        kern<<<plan.grid, plan.block, plan.smem_bytes, stream>>>(mk, mv, dp);
-        return cudaGetLastError();
-    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = plan.grid;
     cfg.blockDim = plan.block;
     cfg.dynamicSmemBytes = plan.smem_bytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    // The grid may be launched while the kernel before it in the stream is
+    // still finishing; it waits (griddepcontrol.wait) before its first global
+    // read, so stream order holds for every input and for the workspace.
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (plan.splits > 1) {
+        attr[n].id = cudaLaunchAttributeCooperative;
+        attr[n].val.cooperative = 1;
+        ++n;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = n;
     return cudaLaunchKernelEx(&cfg, kern, mk, mv, dp);
 }
 

@@ -209,16 +209,17 @@ __global__ void __launch_bounds__(kThreads) flash_ffma_kernel(const AttnParams p
 // tiles of TN = 64.  Thread (ty, tx) of the 32 x 8 grid holds the scores of
 // rows 4*ty .. 4*ty+3 against keys tx, tx+8, .., tx+56 (32 accumulators) and,
 // for the P.V product, the same 4 rows against Dv/8 output columns.  Per four
-// steps along d a thread reads 4 float4 of Q and 8 float4 of K for 128 FMAs.
+// steps along d a thread reads 4 float4 of Q and 8 float4 of K for 128 FMAs;
+// P.V runs on packed f32x2 FMAs (fp32 rounding per lane, half the issue slots).
 //
 // Shared memory (fp32):
 //   Qt[d][row]   Q transposed once per CTA, pre-multiplied by scale*log2(e)
 //   K[key][d]    row stride DQK+4 (an odd number of 16-byte units: the eight
 //                keys tx = 0..7 a quarter-warp reads hit distinct bank groups)
 //   V[key][c]    row stride Dv
-//   Pt[key][row] P transposed; the 16-byte unit of rows 4u..4u+3 sits at unit
-//                u ^ (key & 7), so the stores of eight consecutive keys and the
-//                loads of one key are both conflict-free
+//   Pt[key][row] P transposed, row stride 128+4 (33 16-byte units): the stores
+//                of eight consecutive keys hit distinct bank groups, and the
+//                loads of one key are plain offsets
 // K and V arrive by cp.async: V of tile j while its scores are computed, K of
 // tile j+1 while P.V of tile j runs.
 constexpr int kTM = 128;
@@ -232,7 +233,8 @@ struct TiledSmem {
     static constexpr int KS = DQK + 4;
     static_assert((KS / 4) % 2 == 1, "K row stride must be an odd number of 16-byte units");
     static constexpr int VS = DV;
-    static constexpr int PS = kTM;
+    static constexpr int PS = kTM + 4;
+    static_assert((PS / 4) % 2 == 1, "Pt row stride must be an odd number of 16-byte units");
     static constexpr int k_off = DQK * QS;
     static constexpr int v_off = k_off + kTN * KS;
     static constexpr int p_off = v_off + kTN * VS;
@@ -398,20 +400,26 @@ __global__ void __launch_bounds__(kTThreads, MINB) flash_tiled_f32_kernel(const 
             }
         }
 
+        // Rows past the group (zero Q, never stored) need no masking; a full
+        // unmasked tile needs none at all.
+        if (MASK != 0 || nvalid < kTN) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int jj = tx + 8 * k;
+                    const int64_t j = kt + jj;
+                    bool keep = jj < nvalid;
+                    if (MASK == 1 && keep)
+                        s[i][k] += __ldg(reinterpret_cast<const float*>(p.mask) + moff[i] + j * p.sm[3]) * log2e;
+                    if (MASK == 2 && keep)
+                        keep = __ldg(reinterpret_cast<const uint8_t*>(p.mask) + moff[i] + j * p.sm[3]) != 0;
+                    if (MASK == 3) keep = keep && j <= qi[i] + p.Lk - p.Lq;
+                    if (!keep) s[i][k] = -INFINITY;
+                }
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int jj = tx + 8 * k;
-                const int64_t j = kt + jj;
-                bool keep = rok[i] && jj < nvalid;
-                if (MASK == 1 && keep)
-                    s[i][k] += __ldg(reinterpret_cast<const float*>(p.mask) + moff[i] + j * p.sm[3]) * log2e;
-                if (MASK == 2 && keep)
-                    keep = __ldg(reinterpret_cast<const uint8_t*>(p.mask) + moff[i] + j * p.sm[3]) != 0;
-                if (MASK == 3) keep = keep && j <= qi[i] + p.Lk - p.Lq;
-                if (!keep) s[i][k] = -INFINITY;
-            }
             float mx = fmaxf(fmaxf(fmaxf(s[i][0], s[i][1]), fmaxf(s[i][2], s[i][3])),
                              fmaxf(fmaxf(s[i][4], s[i][5]), fmaxf(s[i][6], s[i][7])));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -432,8 +440,8 @@ __global__ void __launch_bounds__(kTThreads, MINB) flash_tiled_f32_kernel(const 
             for (int n = 0; n < C::NC; ++n) o[i][n] *= alpha;
         }
 #pragma unroll
-        for (int k = 0; k < 8; ++k)   // key tx + 8k: its unit swizzle is tx
-            *reinterpret_cast<float4*>(Pt + (tx + 8 * k) * S::PS + 4 * (ty ^ tx)) =
+        for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<float4*>(Pt + (tx + 8 * k) * S::PS + 4 * ty) =
                 make_float4(s[0][k], s[1][k], s[2][k], s[3][k]);
 
         cp_async_wait<0>();   // V of this tile
@@ -441,13 +449,27 @@ __global__ void __launch_bounds__(kTThreads, MINB) flash_tiled_f32_kernel(const 
         if (kt + kTN < k_end)
             tiled_issue_rows<DQK, S::KS>(Ks, kg + (kt + kTN) * p.sk[2], p.sk[2], (int)min((int64_t)kTN, k_end - kt - kTN));
 
-#pragma unroll 4
+#pragma unroll 8
         for (int j = 0; j < kTN; ++j) {
-            const float4 pf = *reinterpret_cast<const float4*>(Pt + j * S::PS + 4 * (ty ^ (j & 7)));
+            const float4 pf = *reinterpret_cast<const float4*>(Pt + j * S::PS + 4 * ty);
             float vv[C::NC];
             tiled_load_v<DV>(vv, Vs + j * S::VS, tx);
+            // packed f32x2 FMAs over column pairs (each lane an ordinary fp32 FMA):
+            // half the issue slots of scalar FFMA for the same arithmetic
+            const uint64_t pp[4] = {f2_pack(pf.x, pf.x), f2_pack(pf.y, pf.y), f2_pack(pf.z, pf.z),
+                                    f2_pack(pf.w, pf.w)};
 #pragma unroll
-            for (int n = 0; n < C::NC; ++n) {
+            for (int n = 0; n + 1 < C::NC; n += 2) {
+                const uint64_t v2 = f2_pack(vv[n], vv[n + 1]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint64_t r = f2_fma(pp[i], v2, f2_pack(o[i][n], o[i][n + 1]));
+                    o[i][n] = f2_lo(r);
+                    o[i][n + 1] = f2_hi(r);
+                }
+            }
+            if constexpr (C::NC % 2 == 1) {
+                constexpr int n = C::NC - 1;
                 o[0][n] = fmaf(pf.x, vv[n], o[0][n]);
                 o[1][n] = fmaf(pf.y, vv[n], o[1][n]);
                 o[2][n] = fmaf(pf.z, vv[n], o[2][n]);

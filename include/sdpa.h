@@ -17,7 +17,11 @@
  *     ("full") path, as in that issue's section "Current routing";
  *   - head dims: Dqk in {64, 72, 80, 96, 128, 192, 256, 512} with Dv == Dqk,
  *     plus (Dqk, Dv) = (192, 128) (same section; head dim 72 from MLX PR #4330
- *     "Support head dimension 72 in Metal full attention");
+ *     "Support head dimension 72 in Metal full attention"), plus (40, 32):
+ *     absorbed multi-head latent attention on the small MLA fixture of mlxcel
+ *     issue #1065, section "Why this is a precision problem" (keys = 32 latent
+ *     + 8 rope columns, values = the 32 latent columns, so v may point at k
+ *     with k's strides); these dims run on the CUDA-core kernels;
  *   - masks: none, additive, boolean, causal (MLX PR #4330, "Proposed changes").
  *
  * Layout is never inferred from a tensor's shape: every tensor is passed as a

@@ -56,6 +56,11 @@ bool dims_supported(int64_t Dqk, int64_t Dv) {
     switch (Dqk) {
         case 64: case 72: case 80: case 96: case 128: case 256: case 512: return Dv == Dqk;
         case 192: return Dv == 128;
+        // absorbed multi-head latent attention on the small MLA fixture of mlxcel
+        // issue #1065 ("Why this is a precision problem": kv_lora_rank 32,
+        // qk_rope_head_dim 8): keys are [latent | rope] = 40 wide, values are
+        // the 32 latent columns (V may alias K through its strides)
+        case 40: return Dv == 32;
         default: return false;
     }
 }

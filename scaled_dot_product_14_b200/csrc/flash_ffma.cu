@@ -89,15 +89,27 @@ __global__ void __launch_bounds__(kThreads) flash_ffma_kernel(const AttnParams p
     const int64_t hq = hkv * G + (row_ok ? gr / p.Lq : 0);
     const int64_t qi = row_ok ? gr % p.Lq : 0;
 
-    // Q rows, pre-multiplied by scale*log2(e).  Rows of one tile may belong to two heads.
-    for (int rr = 0; rr < kRT; ++rr) {
-        const int64_t g2 = row0 + rr;
-        if (g2 < R) {
-            const int64_t h2 = hkv * G + g2 / p.Lq, i2 = g2 % p.Lq;
-            load_rows_to_float<T>(Qs + rr * S::QS, S::QS, qg + b * p.sq[0] + h2 * p.sq[1] + i2 * p.sq[2], 0, 1, 1,
-                                  DQK, p.scale_log2);
-        } else {
-            for (int d = tid; d < DQK; d += kThreads) Qs[rr * S::QS + d] = 0.f;
+    // Q rows, pre-multiplied by scale*log2(e).  Rows of one tile may belong to two
+    // heads.  One pass over every (row, 16-byte chunk), so all loads are in flight
+    // together rather than one row's latency after another.
+    {
+        constexpr int V = 16 / sizeof(T);
+        constexpr int CH = DQK / V;
+        for (int idx = tid; idx < kRT * CH; idx += kThreads) {
+            const int rr = idx / CH, c = idx % CH;
+            const int64_t g2 = row0 + rr;
+            float* d = Qs + rr * S::QS + c * V;
+            if (g2 < R) {
+                const int64_t h2 = hkv * G + g2 / p.Lq, i2 = g2 % p.Lq;
+                const uint4 raw =
+                    __ldg(reinterpret_cast<const uint4*>(qg + b * p.sq[0] + h2 * p.sq[1] + i2 * p.sq[2] + c * V));
+                const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+                for (int u = 0; u < V; ++u) d[u] = Elem<T>::to_float(e[u]) * p.scale_log2;
+            } else {
+#pragma unroll
+                for (int u = 0; u < V; ++u) d[u] = 0.f;
+            }
         }
     }
 
@@ -517,6 +529,7 @@ cudaError_t launch_tiled(const AttnParams& p, const LaunchPlan& plan, cudaStream
 // Head dims of the tiled kernel (Dv <= 128 keeps the accumulators in registers).
 size_t tiled_smem_for(int64_t Dqk, int64_t Dv) {
     switch (Dqk * 1000 + Dv) {
+        case 40032: return TiledSmem<40, 32>::bytes;
         case 64064: return TiledSmem<64, 64>::bytes;
         case 72072: return TiledSmem<72, 72>::bytes;
         case 80080: return TiledSmem<80, 80>::bytes;
@@ -529,6 +542,7 @@ size_t tiled_smem_for(int64_t Dqk, int64_t Dv) {
 
 cudaError_t launch_tiled_dims(const AttnParams& p, const LaunchPlan& plan, cudaStream_t s) {
     switch (p.Dqk * 1000 + p.Dv) {
+        case 40032: return launch_tiled<40, 32>(p, plan, s);
         case 64064: return launch_tiled<64, 64>(p, plan, s);
         case 72072: return launch_tiled<72, 72>(p, plan, s);
         case 80080: return launch_tiled<80, 80>(p, plan, s);
@@ -551,6 +565,7 @@ cudaError_t launch_one(const AttnParams& p, const LaunchPlan& plan, cudaStream_t
 template <typename T>
 cudaError_t launch_typed(const AttnParams& p, const LaunchPlan& plan, cudaStream_t s) {
     switch (p.Dqk * 1000 + p.Dv) {
+        case 40032: return launch_one<T, 40, 32>(p, plan, s);
         case 64064: return launch_one<T, 64, 64>(p, plan, s);
         case 72072: return launch_one<T, 72, 72>(p, plan, s);
         case 80080: return launch_one<T, 80, 80>(p, plan, s);
@@ -565,6 +580,7 @@ cudaError_t launch_typed(const AttnParams& p, const LaunchPlan& plan, cudaStream
 
 size_t smem_for(int64_t Dqk, int64_t Dv) {
     switch (Dqk * 1000 + Dv) {
+        case 40032: return FfmaSmem<40, 32>::bytes;
         case 64064: return FfmaSmem<64, 64>::bytes;
         case 72072: return FfmaSmem<72, 72>::bytes;
         case 80080: return FfmaSmem<80, 80>::bytes;

@@ -47,7 +47,8 @@ def sup(B=1, Hq=32, Hkv=8, Lq=1, Lk=4096, Dqk=256, Dv=None, layout="bhld", mask_
     return S.sdpa_supported(B, Hq, Hkv, Lq, Lk, Dqk, Dv, st, mask_kind, mask_strides, dtype)
 
 
-@pytest.mark.parametrize("D,Dv", [(64, 64), (72, 72), (80, 80), (96, 96), (128, 128), (192, 128), (256, 256), (512, 512)])
+@pytest.mark.parametrize("D,Dv", [(64, 64), (72, 72), (80, 80), (96, 96), (128, 128), (192, 128), (256, 256), (512, 512),
+                                  (40, 32)])
 @pytest.mark.parametrize("dtype", [0, 1, 2])
 @pytest.mark.parametrize("layout", ["bhld", "blhd"])
 def test_supported_head_dims_both_paths(lib, D, Dv, dtype, layout):
@@ -57,7 +58,8 @@ def test_supported_head_dims_both_paths(lib, D, Dv, dtype, layout):
     assert sup(Lq=8192, Lk=8192, Dqk=D, Dv=Dv, dtype=dtype, layout=layout) == (0, S.SDPA_PATH_PREFILL)
 
 
-@pytest.mark.parametrize("D,Dv", [(32, 32), (48, 48), (192, 192), (128, 64), (256, 128), (512, 256), (100, 100)])
+@pytest.mark.parametrize("D,Dv", [(32, 32), (48, 48), (192, 192), (128, 64), (256, 128), (512, 256), (100, 100),
+                                  (40, 40), (32, 40), (40, 24)])
 def test_unsupported_head_dims_are_errors(lib, D, Dv):
     assert sup(Dqk=D, Dv=Dv)[0] == 2
 

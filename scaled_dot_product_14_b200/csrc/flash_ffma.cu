@@ -17,7 +17,6 @@
 // (running max and sum in the log2 domain, fp32).
 #include <cuda_runtime.h>
 #include <math.h>
-#include <stdlib.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -602,7 +601,7 @@ bool ffma_supported(int dtype, int64_t Dqk, int64_t Dv) {
 LaunchPlan ffma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev, bool split_keys) {
     LaunchPlan plan{};
     const size_t tiled = tiled_smem_for(p.Dqk, p.Dv);
-    if (!split_keys && dtype == 0 && tiled != 0 && !getenv("SDPA_FFMA_UNTILED")) {
+    if (!split_keys && dtype == 0 && tiled != 0) {
         // fp32 prefill: the register-tiled kernel, one CTA per 128 group rows
         const int64_t R = (int64_t)p.group * p.Lq;
         plan.grid = dim3((unsigned)((R + kTM - 1) / kTM), (unsigned)p.Hkv, (unsigned)p.B);

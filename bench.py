@@ -160,18 +160,24 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- distributed
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend="nccl"):
+    """One process per GPU, ranks from the launcher's RANK / LOCAL_RANK / WORLD_SIZE.
+    NCCL between GPUs; gloo runs the same plumbing on host memory only."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if n_gpus != world:
+        print(f"note: --gpus {n_gpus} but WORLD_SIZE={world}; using {world} rank(s)", file=sys.stderr)
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -187,9 +193,16 @@ def max_over_ranks(x, world):
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_gbs(world, bytes_per_step, steps, ms):
+    """Whole-job throughput: every rank moves bytes_per_step per step (weak scaling),
+    over the slowest rank's time."""
+    return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -280,7 +293,7 @@ def run_ours(args, peaks):
     ms = ev0.elapsed_time(ev1)
     ms = max_over_ranks(ms, world)
     ms_per_step = ms / steps_run
-    value = world * bytes_per_step * steps_run / (ms * 1e-3) / 1e9
+    value = aggregate_gbs(world, bytes_per_step, steps_run, ms)
 
     # dominant kernel alone: the library brackets each kernel with events on the
     # launching stream; a GPU-side sleep queued first lets every profiled launch
@@ -382,7 +395,7 @@ def e2e(S, c, t, out, stream, args, world):
         e1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world)
-    val = world * decode_bytes(decode_workload(args.kl)) * n / (ms * 1e-3) / 1e9
+    val = aggregate_gbs(world, decode_bytes(decode_workload(args.kl)), n, ms)
     return {"value": round(val, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": n, "ms_per_step": round(ms / n, 4)}
 

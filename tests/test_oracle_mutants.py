@@ -25,6 +25,12 @@ MUTANTS = {
     "no_normalise": ("for (int64_t e = 0; e < Dv; ++e) o[e] /= l;", ";"),
     "mask_lq_index_dropped": ("i * (mask_st ? mask_st[2] : 0)", "0"),
     "bf16_low_half": ("uint32_t bits = ((uint32_t)b) << 16;", "uint32_t bits = ((uint32_t)b) << 15;"),
+    "mask_scaled": ("sj += oracle_load(mask, midx, dtype);", "sj += scale * oracle_load(mask, midx, dtype);"),
+    "causal_off_by_one": ("if (j > i + (Lk - Lq)) sj = -INFINITY;", "if (j >= i + (Lk - Lq)) sj = -INFINITY;"),
+    "v_from_kv_head_zero": ("g * sv[1] + j * sv[2]", "0 * sv[1] + j * sv[2]"),
+    "q_from_kv_head": ("b * sq[0] + h * sq[1]", "b * sq[0] + g * sq[1]"),
+    "dot_over_dv": ("for (int64_t d = 0; d < Dqk; ++d) {", "for (int64_t d = 0; d < (Dv < Dqk ? Dv : Dqk); ++d) {"),
+    "empty_row_guard_dropped": ("if (l > 0.0) {", "{"),
 }
 
 
@@ -44,6 +50,15 @@ def _pins_hold() -> bool:
                 c.mask.reshape(c.Lq, c.Lk)[:, 0] = 1
             if np.abs(full(O, c) - _torch_ref(c)).max() > 1e-12:
                 return False
+        # Dqk != Dv: the score sum runs over Dqk, the output over Dv
+        c = I.make_case(79, 1, 4, 2, 5, 7, 192, 128, dtype=I.BF16)
+        if np.abs(full(O, c) - _torch_ref(c)).max() > 1e-12:
+            return False
+        # bottom-right causal with Lq > Lk: queries 0..2 see no key and give exact zeros
+        c = I.make_case(80, 1, 2, 2, 6, 3, 64, dtype=I.F32, mask="causal")
+        o = full(O, c)
+        if not (np.all(o[:, :, :3] == 0.0) and np.isfinite(o).all()):
+            return False
         # causal with Lq != Lk: the query chunk [3, 4) of a Lq = 4 problem
         c = I.make_case(78, 1, 2, 2, 4, 9, 64, dtype=I.F32, mask="causal")
         last = full(O, c)[:, :, 3:4]

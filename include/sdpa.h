@@ -39,6 +39,12 @@
  *
  * Threading: the functions are thread-safe.  Execution is asynchronous on the
  * caller's stream; validation is synchronous and happens before any launch.
+ * The fp16/bf16 decode kernel is launched with programmatic dependent launch
+ * allowed: its blocks may start while the previous kernel of the stream is
+ * still running, but none touches global memory before that kernel has
+ * completed (griddepcontrol.wait), so stream order holds for every input and
+ * output.  A later kernel launched the same way may likewise start early and
+ * must wait the same way before it reads this call's output.
  * There is no fallback path of any kind: a case the kernels do not cover is
  * rejected with an error status and nothing is launched.
  */

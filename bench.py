@@ -364,9 +364,65 @@ def run_prefill_only(args, peaks):
         print(json.dumps(entry), flush=True)
 
 
+def parse_cpulist(text):
+    """A sysfs CPU list ("0-3,8,10-11") as a set of CPU numbers."""
+    cpus = set()
+    for part in text.strip().split(","):
+        part = part.strip()
+        if not part:
+            continue
+        if "-" in part:
+            a, b = part.split("-")
+            cpus.update(range(int(a), int(b) + 1))
+        else:
+            cpus.add(int(part))
+    return cpus
+
+
+def gpu_local_cpus(device):
+    """The CPUs of the GPU's NUMA node (sysfs local_cpulist of its PCI function)
+    that this process may run on, or None when that cannot be read."""
+    import torch
+    try:
+        pr = torch.cuda.get_device_properties(device)
+        path = (f"/sys/bus/pci/devices/{pr.pci_domain_id:04x}:{pr.pci_bus_id:02x}:"
+                f"{pr.pci_device_id:02x}.0/local_cpulist")
+        with open(path) as f:
+            cpus = parse_cpulist(f.read()) & os.sched_getaffinity(0)
+        return cpus or None
+    except Exception:
+        return None
+
+
 def e2e(S, c, t, out, stream, args, world):
     """Same metric through the C ABI from pinned host buffers: H2D of the step's
-    inputs, the call, D2H of the output, all inside the timed region."""
+    inputs, the call, D2H of the output, all inside the timed region.  The host
+    buffers are allocated and driven from the CPUs next to the GPU (the process's
+    CPU affinity is restored afterwards)."""
+    import torch
+    saved = os.sched_getaffinity(0)
+    local_cpus = gpu_local_cpus(torch.cuda.current_device())
+    pinned = False
+    if local_cpus:
+        try:
+            os.sched_setaffinity(0, local_cpus)
+            pinned = True
+        except OSError:
+            pass
+    try:
+        res = _e2e_timed(S, c, t, out, stream, args, world)
+    finally:
+        if pinned:
+            try:
+                os.sched_setaffinity(0, saved)
+            except OSError:
+                pass
+    res["host_cpus"] = (f"{len(local_cpus)} CPUs of the GPU's NUMA node" if pinned
+                        else "process default (GPU NUMA node not found)")
+    return res
+
+
+def _e2e_timed(S, c, t, out, stream, args, world):
     import torch
     host = {k: v.cpu().pin_memory() for k, v in t.items() if v is not None}
     dev = {k: torch.empty_like(v) for k, v in t.items() if v is not None}

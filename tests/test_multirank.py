@@ -80,3 +80,12 @@ def test_reference_arm_on_a_nonzero_rank_exits_quietly():
                         "--warmup", "1"], env=env, capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_cpulist_parsing():
+    """The e2e leg reads the GPU's NUMA-local CPUs from a sysfs CPU list."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.parse_cpulist("0-3,8,10-11\n") == {0, 1, 2, 3, 8, 10, 11}
+    assert bench.parse_cpulist("5") == {5}
+    assert bench.parse_cpulist("") == set()

@@ -364,6 +364,15 @@ def run_prefill_only(args, peaks):
         print(json.dumps(entry), flush=True)
 
 
+def usable_cpus():
+    """CPUs this process may run on (its affinity set), which is what the oracle's
+    thread pool can actually use."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def parse_cpulist(text):
     """A sysfs CPU list ("0-3,8,10-11") as a set of CPU numbers."""
     cpus = set()
@@ -565,7 +574,7 @@ def cpu_baseline(w, seconds):
     oracle.build()
     c = I.make_case(w["seed"], w["B"], w["Hq"], w["Hkv"], w["Lq"], w["Lk"], w["Dqk"], w["Dv"],
                     dtype=I.DTYPE_BY_NAME[w["dtype"]], mask=w["mask"], layout=w["layout"])
-    threads = os.cpu_count() or 1
+    threads = usable_cpus()
     n, t0 = 0, time.time()
     while True:
         oracle.sdpa_rows(c.q, c.k, c.v, B=c.B, Hq=c.Hq, Hkv=c.Hkv, Lq=c.Lq, Lk=c.Lk, Dqk=c.Dqk, Dv=c.Dv,
@@ -592,7 +601,7 @@ def run_reference(args):
     w = decode_workload(args.kl)
     c = I.make_case(w["seed"], w["B"], w["Hq"], w["Hkv"], w["Lq"], w["Lk"], w["Dqk"], w["Dv"],
                     dtype=I.DTYPE_BY_NAME[w["dtype"]], mask=w["mask"], layout=w["layout"])
-    threads = os.cpu_count() or 1
+    threads = usable_cpus()
 
     def step():
         oracle.sdpa_rows(c.q, c.k, c.v, B=c.B, Hq=c.Hq, Hkv=c.Hkv, Lq=c.Lq, Lk=c.Lk, Dqk=c.Dqk, Dv=c.Dv,

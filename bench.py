@@ -5,9 +5,14 @@ Headline workload (one step = one decode call through the C ABI):
   decode ("vector" path of MLX issue #3885): bf16, B=1, qL=1, kL=4096,
   Hq=32, Hkv=8 (GQA 4), D=256, additive mask [1,1,1,kL] U(-1,0) with the last
   10% of keys -inf; Q/K/V ~ N(0,1) seeded.
-Metric: decode KV GB/s = algorithmic bytes (K+V+Q+O footprint) / time; the
-prefill TFLOP/s of the head-dim-72 and head-dim-512 prefill workloads are
-reported alongside in "prefill".
+Metric: decode KV GB/s = algorithmic bytes (K+V+Q+O footprint) / time.  Reported
+alongside:
+  "prefill": TFLOP/s of the head-dim-72 and head-dim-512 bf16 prefill workloads
+             and of one fp32 prefill row (FFMA roofline);
+  "mla_decode": microseconds per absorbed-MLA decode call on the small latent
+             fixture (fp32 and bf16);
+  "e2e": the headline metric through the C ABI from pinned host buffers;
+  "cpu_baseline": the float64 oracle on the host's cores.
 
 Timing: W warm-up steps, then K steps bracketed by a barrier and
 torch.cuda.synchronize() on both sides, CUDA events on the launching stream,

@@ -30,7 +30,7 @@ _SRC = os.path.join(_HERE, "sdpa_oracle.c")
 _LIB = os.path.join(_HERE, "_liboracle_sdpa.so")
 
 F32, F16, BF16 = 0, 1, 2
-MASK_NONE, MASK_ADDITIVE, MASK_BOOL, MASK_CAUSAL = 0, 1, 2, 3
+MASK_NONE, MASK_ADDITIVE, MASK_BOOL, MASK_CAUSAL, MASK_SLIDING = 0, 1, 2, 3, 4
 
 _lib = None
 _lock = threading.Lock()
@@ -55,7 +55,7 @@ def _load():
             i64, p = ctypes.c_int64, ctypes.c_void_p
             lib.oracle_sdpa_rows.restype = ctypes.c_int
             lib.oracle_sdpa_rows.argtypes = [p, p, p, i64, i64, i64, i64, i64, i64, i64, p,
-                                             ctypes.c_double, ctypes.c_int, p, p, ctypes.c_int,
+                                             ctypes.c_double, ctypes.c_int, p, p, i64, ctypes.c_int,
                                              p, i64, p, p]
             lib.oracle_version.restype = ctypes.c_int
             _lib = lib
@@ -68,14 +68,14 @@ def _ptr(a):
 
 def sdpa_rows(q, k, v, *, B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, scale, dtype,
               mask_kind=MASK_NONE, mask=None, mask_strides=(0, 0, 0, 0), rows=None,
-              threads=None, want_probs=False):
+              threads=None, want_probs=False, window=0):
     """Attention for selected query rows, in float64.
 
     q, k, v, mask: 1-D numpy storage buffers (float32 for fp32, uint16 bit
     patterns for fp16 / bf16, uint8 for a boolean mask); ``strides`` holds the
     12 element strides (b, h, l, d) of q, k and v into those buffers.
     ``rows`` is an (n, 3) int64 array of (b, h, i); None means every row in
-    (b, h, i) order.  Returns (n, Dv) float64 (and (n, Lk) weights if asked).
+    (b, h, i) order.  ``window``: the key count of the sliding-window mask kind.  Returns (n, Dv) float64 (and (n, Lk) weights if asked).
     """
     lib = _load()
     if rows is None:
@@ -96,7 +96,7 @@ def sdpa_rows(q, k, v, *, B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, scale, dtype,
         pr = probs[lo:hi] if probs is not None else None
         rc = lib.oracle_sdpa_rows(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Lq, Lk, Dqk, Dv,
                                   _ptr(st), float(scale), int(mask_kind), _ptr(mask), _ptr(mst),
-                                  int(dtype), _ptr(rows[lo:hi]), hi - lo, _ptr(o), _ptr(pr))
+                                  int(window), int(dtype), _ptr(rows[lo:hi]), hi - lo, _ptr(o), _ptr(pr))
         if rc != 0:
             raise ValueError("oracle rejected its arguments")
 
@@ -111,9 +111,9 @@ def sdpa_rows(q, k, v, *, B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, scale, dtype,
 
 
 def sdpa_full(q, k, v, *, B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, scale, dtype,
-              mask_kind=MASK_NONE, mask=None, mask_strides=(0, 0, 0, 0), threads=None):
+              mask_kind=MASK_NONE, mask=None, mask_strides=(0, 0, 0, 0), threads=None, window=0):
     """Every row; returns float64 [B, Hq, Lq, Dv]."""
     o = sdpa_rows(q, k, v, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, Dqk=Dqk, Dv=Dv, strides=strides,
                   scale=scale, dtype=dtype, mask_kind=mask_kind, mask=mask,
-                  mask_strides=mask_strides, threads=threads)
+                  mask_strides=mask_strides, threads=threads, window=window)
     return o.reshape(B, Hq, Lq, Dv)

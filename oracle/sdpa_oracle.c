@@ -24,12 +24,20 @@
  *   MLX PR #4330 ("Support head dimension 72 in Metal full attention"),
  *   "Proposed changes": masks are none, additive, boolean or causal.
  *
+ *   MLX issue #3885, "Current routing": Gemma 4's hybrid layout has sliding
+ *   (local) attention layers next to its global ones.  The pages name the
+ *   layers but not their rule; the reading taken here is causal attention
+ *   limited to a window of the `window` most recent keys.
+ *
  * Readings taken where the pages are silent (each is also a test):
  *   - additive mask: added after scaling: s_j = scale * (q . k_j) + mask_ij;
  *     entries may be -inf;
  *   - boolean mask: nonzero = attend, zero = the key is removed (-inf);
  *   - causal with Lq != Lk: bottom-right alignment, key j is visible to
  *     query i iff j <= i + (Lk - Lq); with Lq == Lk this is plain causal;
+ *   - sliding window of W keys: with the same alignment, key j is visible to
+ *     query i iff i + (Lk - Lq) - W < j <= i + (Lk - Lq): the W most recent
+ *     keys up to the query's own position (W >= Lk is plain causal);
  *   - a row whose every key is removed outputs zeros (no NaN).
  *
  * Every element is widened exactly to double (fp32, fp16 and bf16 values are
@@ -42,7 +50,8 @@
 #include <string.h>
 
 enum { ORACLE_F32 = 0, ORACLE_F16 = 1, ORACLE_BF16 = 2 };
-enum { ORACLE_MASK_NONE = 0, ORACLE_MASK_ADDITIVE = 1, ORACLE_MASK_BOOL = 2, ORACLE_MASK_CAUSAL = 3 };
+enum { ORACLE_MASK_NONE = 0, ORACLE_MASK_ADDITIVE = 1, ORACLE_MASK_BOOL = 2, ORACLE_MASK_CAUSAL = 3,
+       ORACLE_MASK_SLIDING = 4 };
 
 /* IEEE binary16 -> double, from the format's definition
  * (1 sign bit, 5 exponent bits with bias 15, 10 fraction bits). */
@@ -82,6 +91,7 @@ static double oracle_load(const void* base, int64_t idx, int dtype) {
  * strides    : 12 element strides, (b, h, l, d) for q, then k, then v.
  * mask       : for ADDITIVE, storage dtype `dtype`; for BOOL, uint8.
  * mask_st    : 4 element strides (b, h, lq, lk) of the mask; 0 broadcasts.
+ * window     : for SLIDING, the number of most recent keys a query sees (>= 1).
  * rows       : nrows triples (b, h, i) naming the query rows to compute.
  * out        : nrows * Dv doubles, row-major.
  * probs      : optional (may be NULL): nrows * Lk doubles, the normalised
@@ -91,9 +101,10 @@ static double oracle_load(const void* base, int64_t idx, int dtype) {
 int oracle_sdpa_rows(const void* q, const void* k, const void* v,
                      int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk,
                      int64_t Dqk, int64_t Dv, const int64_t* strides, double scale,
-                     int mask_kind, const void* mask, const int64_t* mask_st, int dtype,
+                     int mask_kind, const void* mask, const int64_t* mask_st, int64_t window, int dtype,
                      const int64_t* rows, int64_t nrows, double* out, double* probs) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Lq < 0 || Lk < 0 || Dqk <= 0 || Dv <= 0) return -1;
+    if (mask_kind == ORACLE_MASK_SLIDING && window < 1) return -1;
     if (Hq % Hkv != 0) return -1;
     if (dtype < ORACLE_F32 || dtype > ORACLE_BF16) return -1;
     const int64_t n_rep = Hq / Hkv;
@@ -125,6 +136,9 @@ int oracle_sdpa_rows(const void* q, const void* k, const void* v,
                 if (((const uint8_t*)mask)[midx] == 0) sj = -INFINITY;
             } else if (mask_kind == ORACLE_MASK_CAUSAL) {
                 if (j > i + (Lk - Lq)) sj = -INFINITY;
+            } else if (mask_kind == ORACLE_MASK_SLIDING) {
+                const int64_t own = i + (Lk - Lq);        /* the query's own key position */
+                if (j > own || j <= own - window) sj = -INFINITY;
             }
             s[j] = sj;
         }
@@ -158,4 +172,4 @@ int oracle_sdpa_rows(const void* q, const void* k, const void* v,
 }
 
 /* Version tag so the Python side can check it loaded this file's build. */
-int oracle_version(void) { return 1; }
+int oracle_version(void) { return 2; }

@@ -25,7 +25,7 @@ F32, F16, BF16 = 0, 1, 2
 DTYPE_NAMES = {F32: "f32", F16: "f16", BF16: "bf16"}
 DTYPE_BY_NAME = {"f32": F32, "fp32": F32, "f16": F16, "fp16": F16, "bf16": BF16}
 ELEM_SIZE = {F32: 4, F16: 2, BF16: 2}
-MASK_NONE, MASK_ADDITIVE, MASK_BOOL, MASK_CAUSAL = 0, 1, 2, 3
+MASK_NONE, MASK_ADDITIVE, MASK_BOOL, MASK_CAUSAL, MASK_SLIDING = 0, 1, 2, 3, 4
 
 
 # ----------------------------------------------------------------------------- dtype storage
@@ -112,6 +112,7 @@ class Case:
     mask_strides: tuple = (0, 0, 0, 0)
     layout: str = "bhld"
     meta: dict = field(default_factory=dict)
+    window: int = 0                     # sliding-window mask: keys each query sees (0 = not that kind)
 
     @property
     def all_strides16(self):
@@ -125,11 +126,11 @@ def default_scale(Dqk: int) -> float:
 
 def make_case(seed: int, B: int, Hq: int, Hkv: int, Lq: int, Lk: int, Dqk: int, Dv: int | None = None,
               dtype: int = BF16, mask: str = "none", layout: str = "bhld", p_keep: float = 0.9,
-              scale: float | None = None) -> Case:
+              scale: float | None = None, window: int = 0) -> Case:
     """Seeded N(0,1) case.  mask in {"none", "causal", "decode_additive",
     "additive" ([B,1,Lq,Lk] U(-1,0)), "additive_bcast" ([1,1,Lq,Lk]), "additive_full" ([B,Hq,Lq,Lk]),
     "bool" ([1,1,Lq,Lk]),
-    "bool_full" ([B,Hq,Lq,Lk])}."""
+    "bool_full" ([B,Hq,Lq,Lk]), "sliding" (causal limited to the `window` most recent keys)}."""
     Dv = Dqk if Dv is None else Dv
     rng = np.random.default_rng(seed)
     qf = rng.standard_normal((B, Hq, Lq, Dqk), dtype=np.float32)
@@ -144,6 +145,10 @@ def make_case(seed: int, B: int, Hq: int, Hkv: int, Lq: int, Lk: int, Dqk: int, 
     mk, mbuf, mst = MASK_NONE, None, (0, 0, 0, 0)
     if mask == "causal":
         mk = MASK_CAUSAL
+    elif mask == "sliding":
+        if window < 1:
+            raise ValueError("the sliding-window mask needs window >= 1")
+        mk = MASK_SLIDING
     elif mask == "decode_additive":
         m = rng.uniform(-1.0, 0.0, size=(Lk,)).astype(np.float32)
         n_inf = int(np.floor(0.1 * Lk))
@@ -169,7 +174,7 @@ def make_case(seed: int, B: int, Hq: int, Hkv: int, Lq: int, Lk: int, Dqk: int, 
         raise ValueError(mask)
     return Case(B, Hq, Hkv, Lq, Lk, Dqk, Dv, dtype, q, k, v, strides, out_strides,
                 default_scale(Dqk) if scale is None else float(np.float32(scale)),
-                mk, mbuf, mst, layout, {"seed": seed, "mask": mask})
+                mk, mbuf, mst, layout, {"seed": seed, "mask": mask}, window if mk == MASK_SLIDING else 0)
 
 
 def sample_rows(seed: int, B: int, Hq: int, Lq: int, n: int, include_edges: bool = True) -> np.ndarray:

@@ -25,7 +25,7 @@ def run(oracle_mod, c: I.Case, rows=None, want_probs=False):
     return oracle_mod.sdpa_rows(c.q, c.k, c.v, B=c.B, Hq=c.Hq, Hkv=c.Hkv, Lq=c.Lq, Lk=c.Lk,
                                 Dqk=c.Dqk, Dv=c.Dv, strides=c.strides, scale=c.scale, dtype=c.dtype,
                                 mask_kind=c.mask_kind, mask=c.mask, mask_strides=c.mask_strides,
-                                rows=rows, want_probs=want_probs)
+                                rows=rows, want_probs=want_probs, window=c.window)
 
 
 def full(oracle_mod, c: I.Case):
@@ -310,3 +310,79 @@ def test_fp32_path_is_not_reduced_precision(oracle_mod):
     precision.  The oracle on fp32 inputs must agree with torch float64 far below it."""
     c = I.make_case(41, 1, 4, 4, 4, 4, 64, dtype=I.F32, mask="causal")
     assert np.abs(full(oracle_mod, c) - _torch_ref(c)).max() < 1e-12 < 2.0 ** -10
+
+
+# --------------------------------------------------------------------------- sliding window
+# The pages name Gemma 4's sliding (local) attention layers (MLX issue #3885,
+# "Current routing") without their rule; the reading pinned here: with the
+# causal bottom-right alignment own = i + Lk - Lq, key j is visible iff
+# own - W < j <= own.
+@pytest.mark.parametrize("Lq,Lk", [(7, 7), (3, 9), (9, 5)])
+def test_window_of_one_returns_the_own_key(oracle_mod, Lq, Lk):
+    """W = 1: each query sees exactly its own (bottom-right aligned) key, so the
+    row is that key's V row exactly; queries whose own position is before key 0
+    see nothing and give zeros."""
+    c = I.make_case(50, 1, 4, 2, Lq, Lk, 64, dtype=I.BF16, mask="sliding", window=1)
+    o, v = full(oracle_mod, c), logical(c, "v")
+    for h in range(4):
+        for i in range(Lq):
+            own = i + Lk - Lq
+            if own < 0:
+                assert np.all(o[0, h, i] == 0.0)
+            else:
+                np.testing.assert_array_equal(o[0, h, i], v[0, h // 2, own])
+
+
+def test_window_of_two_is_a_two_key_softmax(oracle_mod):
+    """W = 2: the row is the softmax-weighted mean of the V rows at own - 1 and
+    own, weights 1 / (1 + e^(s_other - s_self)) worked out per row here."""
+    c = I.make_case(51, 1, 2, 1, 6, 10, 64, dtype=I.F32, mask="sliding", window=2)
+    o, q, k, v = full(oracle_mod, c), logical(c, "q"), logical(c, "k"), logical(c, "v")
+    for h in range(2):
+        for i in range(6):
+            own = i + 4
+            s_prev = c.scale * float(q[0, h, i] @ k[0, 0, own - 1])
+            s_own = c.scale * float(q[0, h, i] @ k[0, 0, own])
+            w_own = 1.0 / (1.0 + math.exp(s_prev - s_own))
+            expect = w_own * v[0, 0, own] + (1.0 - w_own) * v[0, 0, own - 1]
+            assert np.abs(o[0, h, i] - expect).max() <= 1e-12
+
+
+@pytest.mark.parametrize("W", [9, 10, 1000])
+def test_window_covering_every_key_is_causal(oracle_mod, W):
+    c = I.make_case(52, 2, 4, 2, 9, 9, 80, dtype=I.F16, mask="sliding", window=W)
+    import dataclasses
+    causal = dataclasses.replace(c, mask_kind=I.MASK_CAUSAL, window=0)
+    assert np.abs(full(oracle_mod, c) - _torch_ref(causal)).max() <= 1e-12
+
+
+@pytest.mark.parametrize("W", [1, 3, 8])
+@pytest.mark.parametrize("Lq,Lk", [(12, 12), (5, 17)])
+def test_window_matches_torch_with_a_band_matrix(oracle_mod, W, Lq, Lk):
+    """torch float64 SDPA with an explicit boolean band built as a matrix (lower
+    triangle of the shifted causal mask minus the triangle W below it); rows
+    with an empty band are excluded (torch gives NaN there)."""
+    c = I.make_case(53 + W, 2, 4, 2, Lq, Lk, 128, dtype=I.BF16, mask="sliding", window=W)
+    ones = np.ones((Lq, Lk), dtype=bool)
+    band = np.tril(ones, k=Lk - Lq) & ~np.tril(ones, k=Lk - Lq - W)
+    q = torch.from_numpy(logical(c, "q"))
+    k = torch.from_numpy(logical(c, "k")).repeat_interleave(2, dim=1)
+    v = torch.from_numpy(logical(c, "v")).repeat_interleave(2, dim=1)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=torch.from_numpy(band),
+                                                           scale=c.scale).numpy()
+    o = full(oracle_mod, c)
+    rows = band.any(axis=1)
+    assert np.abs(o[:, :, rows] - ref[:, :, rows]).max() <= 1e-12
+    assert np.all(o[:, :, ~rows] == 0.0)
+
+
+def test_window_chunked_queries_equal_unchunked(oracle_mod):
+    """Bottom-right alignment makes a chunk of the last queries see the same
+    keys as in the whole call (mlxcel issue #1065's chunked-prefill check)."""
+    c = I.make_case(54, 1, 2, 2, 8, 20, 64, dtype=I.F32, mask="sliding", window=5)
+    whole = full(oracle_mod, c)
+    for a in range(8):
+        sub = I.make_case(54, 1, 2, 2, 1, 20 - 7 + a, 64, dtype=I.F32, mask="sliding", window=5)
+        sub = with_values(sub, q=logical(c, "q")[:, :, a:a + 1], k=logical(c, "k")[:, :, :20 - 7 + a],
+                          v=logical(c, "v")[:, :, :20 - 7 + a])
+        assert np.abs(full(oracle_mod, sub)[:, :, 0] - whole[:, :, a]).max() <= 1e-12

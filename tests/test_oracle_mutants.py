@@ -31,6 +31,11 @@ MUTANTS = {
     "q_from_kv_head": ("b * sq[0] + h * sq[1]", "b * sq[0] + g * sq[1]"),
     "dot_over_dv": ("for (int64_t d = 0; d < Dqk; ++d) {", "for (int64_t d = 0; d < (Dv < Dqk ? Dv : Dqk); ++d) {"),
     "empty_row_guard_dropped": ("if (l > 0.0) {", "{"),
+    "window_off_by_one": ("if (j > own || j <= own - window) sj = -INFINITY;",
+                          "if (j > own || j < own - window) sj = -INFINITY;"),
+    "window_not_causal": ("if (j > own || j <= own - window) sj = -INFINITY;",
+                          "if (j <= own - window) sj = -INFINITY;"),
+    "window_top_left": ("const int64_t own = i + (Lk - Lq);", "const int64_t own = i;"),
 }
 
 
@@ -66,6 +71,11 @@ def _pins_hold() -> bool:
         sub = I.make_case(78, 1, 2, 2, 1, 9, 64, dtype=I.F32, mask="causal")
         sub = with_values(sub, q=logical(c, "q")[:, :, 3:4], k=logical(c, "k"), v=logical(c, "v"))
         if np.abs(full(O, sub) - last).max() > 1e-12:
+            return False
+        # sliding window of one key, Lq < Lk: every row is its own key's V row
+        c = I.make_case(81, 1, 2, 1, 3, 7, 64, dtype=I.F32, mask="sliding", window=1)
+        o, v = full(O, c), logical(c, "v")
+        if not all(np.array_equal(o[0, h, i], v[0, 0, i + 4]) for h in range(2) for i in range(3)):
             return False
         return True
     except ValueError:

@@ -66,27 +66,51 @@ def decode_workload(kL=4096):
 PREFILL_WORKLOADS = [
     dict(name="prefill bf16 B=1 H=16 L=8192 D=72 no mask [B,L,H,D]", seed=1003, B=1, Hq=16, Hkv=16, Lq=8192,
          Lk=8192, Dqk=72, Dv=72, dtype="bf16", mask="none", layout="blhd"),
+    dict(name="prefill fp16 B=1 H=16 L=8192 D=72 no mask [B,L,H,D]", seed=1003, B=1, Hq=16, Hkv=16, Lq=8192,
+         Lk=8192, Dqk=72, Dv=72, dtype="f16", mask="none", layout="blhd"),
+    dict(name="prefill bf16 B=1 H=16 L=8192 D=72 bool mask [1,1,L,L] p_keep=0.9 [B,L,H,D]", seed=1003, B=1,
+         Hq=16, Hkv=16, Lq=8192, Lk=8192, Dqk=72, Dv=72, dtype="bf16", mask="bool", layout="blhd"),
     dict(name="prefill bf16 B=1 Hq=32 Hkv=4 L=4096 D=512 causal", seed=1002, B=1, Hq=32, Hkv=4, Lq=4096, Lk=4096,
          Dqk=512, Dv=512, dtype="bf16", mask="causal", layout="bhld"),
-    dict(name="prefill fp32 B=2 Hq=32 Hkv=8 L=2048 D=64 no mask (sweep row, FFMA path)", seed=1004, B=2, Hq=32,
-         Hkv=8, Lq=2048, Lk=2048, Dqk=64, Dv=64, dtype="f32", mask="none", layout="bhld"),
+    dict(name="prefill fp32 B=2 Hq=32 Hkv=8 L=2048 D=64 no mask (sweep row, three-term TF32 on tcgen05)",
+         seed=1004, B=2, Hq=32, Hkv=8, Lq=2048, Lk=2048, Dqk=64, Dv=64, dtype="f32", mask="none", layout="bhld"),
+    dict(name="prefill fp32 B=2 Hq=32 Hkv=8 L=2048 D=128 no mask (sweep row, FFMA path)", seed=1004, B=2, Hq=32,
+         Hkv=8, Lq=2048, Lk=2048, Dqk=128, Dv=128, dtype="f32", mask="none", layout="bhld"),
+    dict(name="prefill bf16 B=1 Hq=32 Hkv=16 L=8192 D=256 sliding window 1024 (Gemma-4 sliding-layer shape)",
+         seed=1010, B=1, Hq=32, Hkv=16, Lq=8192, Lk=8192, Dqk=256, Dv=256, dtype="bf16", mask="sliding",
+         window=1024, layout="bhld"),
 ]
 
-# fp32 runs on the CUDA cores (FFMA): peak = SMs x 128 FMA lanes x 2 FLOP x max SM clock
+# fp32 on the CUDA cores (FFMA): peak = SMs x 128 FMA lanes x 2 FLOP x max SM clock
 FFMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# fp32 on the tensor cores (kind::tf32): the measured bf16 peak x the nominal dense
+# tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s); the three-term split issues 3 MMAs per product
+TF32_OVER_BF16 = 1.1 / 2.25
 
 
 def decode_bytes(w):
-    """Algorithmic bytes of one decode call: K+V read once, Q read, O written."""
+    """Algorithmic bytes of one decode call: K+V read once (for a sliding window,
+    only the keys some query's window holds), Q read, O written."""
     e = 2 if w["dtype"] in ("bf16", "f16") else 4
-    kv = w["B"] * w["Hkv"] * w["Lk"] * (w["Dqk"] + w["Dv"])
+    keys = w["Lk"] if w["mask"] != "sliding" else min(w["Lk"], w["window"] + w["Lq"] - 1)
+    kv = w["B"] * w["Hkv"] * keys * (w["Dqk"] + w["Dv"])
     qo = w["B"] * w["Hq"] * w["Lq"] * (w["Dqk"] + w["Dv"])
     return e * (kv + qo)
 
 
+def visible_keys(w):
+    """Keys summed over the query rows of one (batch, head) that the mask leaves visible
+    (every key; half for causal at Lq = Lk; the window's keys for a sliding window)."""
+    Lq, Lk = w["Lq"], w["Lk"]
+    if w["mask"] == "sliding":
+        own = np.arange(Lq, dtype=np.int64) + (Lk - Lq)
+        return int(np.clip(np.minimum(own + 1, w["window"]), 0, None).sum())
+    return Lq * Lk / 2 if w["mask"] == "causal" else Lq * Lk
+
+
 def prefill_flops(w):
-    f = 2.0 * w["B"] * w["Hq"] * w["Lq"] * w["Lk"] * (w["Dqk"] + w["Dv"])
-    return f / 2 if w["mask"] == "causal" else f
+    """Algorithmic FLOPs: 2 (Dqk + Dv) per visible (query, key) pair."""
+    return 2.0 * w["B"] * w["Hq"] * visible_keys(w) * (w["Dqk"] + w["Dv"])
 
 
 def kernel_source_hash(files):
@@ -215,7 +239,8 @@ def device_case(w, rank):
     import torch
     from scaled_dot_product_14_b200 import inputs as I
     c = I.make_case(w["seed"] + 17 * rank, w["B"], w["Hq"], w["Hkv"], w["Lq"], w["Lk"], w["Dqk"], w["Dv"],
-                    dtype=I.DTYPE_BY_NAME[w["dtype"]], mask=w["mask"], layout=w["layout"])
+                    dtype=I.DTYPE_BY_NAME[w["dtype"]], mask=w["mask"], layout=w["layout"],
+                    window=w.get("window", 0))
 
     def dev(a, is_mask=False):
         if is_mask and c.mask_kind == I.MASK_BOOL:
@@ -230,12 +255,88 @@ def device_case(w, rank):
 
 
 def call(S, c, t, k, v, out, stream):
+    if c.window:
+        st = S.sdpa_forward_window(t["q"].data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), c.B, c.Hq, c.Hkv,
+                                   c.Lq, c.Lk, c.Dqk, c.Dv, c.all_strides16, c.scale, c.window, c.dtype, stream)
+        if st != 0:
+            raise S.SdpaError(st, "sdpa_forward_window")
+        return
     st = S.sdpa_forward(t["q"].data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), c.B, c.Hq, c.Hkv, c.Lq, c.Lk,
                         c.Dqk, c.Dv, c.all_strides16, c.scale, c.mask_kind,
                         None if t["mask"] is None else t["mask"].data_ptr(),
                         None if t["mask"] is None else c.mask_strides, c.dtype, stream)
     if st != 0:
         raise S.SdpaError(st)
+
+
+def decode_graph(S, c, t, copies, steps, stream):
+    """A CUDA graph of exactly `steps` C-ABI decode calls, call i on K/V copy i % copies."""
+    import torch
+    ks = [t["k"]] + [t["k"].clone() for _ in range(copies - 1)]
+    vs = [t["v"]] + [t["v"].clone() for _ in range(copies - 1)]
+    out = torch.empty(c.B * c.Hq * c.Lq * c.Dv, dtype=t["q"].dtype, device="cuda")
+    sp = stream.cuda_stream
+    with torch.cuda.stream(stream):
+        call(S, c, t, ks[0], vs[0], out, sp)          # allocates the split-K workspace before capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(steps):
+            call(S, c, t, ks[i % copies], vs[i % copies], out, sp)
+    torch.cuda.synchronize()
+    return graph, ks, vs, out
+
+
+def time_decode(S, w, rank, world, stream, steps, warmup, soak, clocks=None):
+    """W eager warm-up calls, an untimed soak of graph replays, then one replay
+    of a graph of exactly `steps` calls between events on the launching stream
+    (barrier and synchronize on both sides; max over ranks)."""
+    import torch
+    c, t = device_case(w, rank)
+    kv_bytes = t["k"].numel() * t["k"].element_size() + t["v"].numel() * t["v"].element_size()
+    copies = max(2, math.ceil(2 * L2_BYTES / kv_bytes))
+    graph, ks, vs, out = decode_graph(S, c, t, copies, steps, stream)
+    sp = stream.cuda_stream
+    launches = S.sdpa_last_launch_count()
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            call(S, c, t, ks[i % copies], vs[i % copies], out, sp)
+    if clocks:
+        clocks.start()
+    soak_end = time.time() + soak
+    while time.time() < soak_end:
+        with torch.cuda.stream(stream):
+            graph.replay()
+        stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):            # replay() launches on the current stream
+        ev0.record(stream)
+        graph.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+
+    # each launch alone: the library brackets each kernel with events on the
+    # launching stream; a GPU-side sleep queued first lets the profiled launches
+    # queue up behind it, so they run back to back with no host gaps
+    S.sdpa_profile_enable(True)
+    S.sdpa_profile_collect()
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(20_000_000)          # ~10 ms of GPU time while the host enqueues
+        for r in range(2 * copies):
+            call(S, c, t, ks[r % copies], vs[r % copies], out, sp)
+    torch.cuda.synchronize()
+    prof = S.sdpa_profile_collect()
+    S.sdpa_profile_enable(False)
+    fam = "decode_mma" if c.dtype != 0 else "decode_ffma"
+    n_dec, ms_dec = prof[fam]
+    del graph, ks, vs, out, t
+    return dict(c=c, ms=ms, copies=copies, kv_bytes=kv_bytes, launches=launches, clocks=clk,
+                us_isolated=1e3 * ms_dec / max(n_dec, 1))
 
 
 def run_ours(args, peaks):
@@ -246,78 +347,18 @@ def run_ours(args, peaks):
     if rank == 0 and not os.path.exists(S.LIB_PATH):
         build.build()
     barrier(world)
+    stream = torch.cuda.Stream()
+    steps, warmup = args.steps, max(args.warmup, 3)
 
     w = decode_workload(args.kl)
-    c, t = device_case(w, rank)
     bytes_per_step = decode_bytes(w)
-    kv_bytes = t["k"].numel() * 2 + t["v"].numel() * 2
-    copies = max(2, math.ceil(2 * L2_BYTES / kv_bytes))
-    ks = [t["k"]] + [t["k"].clone() for _ in range(copies - 1)]
-    vs = [t["v"]] + [t["v"].clone() for _ in range(copies - 1)]
-    out = torch.empty(c.B * c.Hq * c.Lq * c.Dv, dtype=t["q"].dtype, device="cuda")
-    stream = torch.cuda.Stream()
-    sp = stream.cuda_stream
-
-    with torch.cuda.stream(stream):
-        call(S, c, t, ks[0], vs[0], out, sp)          # allocates the split-K workspace before capture
-    torch.cuda.synchronize()
-    launches_per_step = S.sdpa_last_launch_count()
-
-    # a graph holding one step per K/V copy; replays cycle through the copies
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for i in range(copies):
-            call(S, c, t, ks[i], vs[i], out, sp)
-    torch.cuda.synchronize()
-    steps = args.steps
-    reps = max(1, math.ceil(steps / copies))
-    steps_run = reps * copies
-
-    clocks = ClockSampler(local)
-    clocks.start()
-    for _ in range(max(args.warmup, 3)):
-        with torch.cuda.stream(stream):
-            call(S, c, t, ks[0], vs[0], out, sp)
-    # untimed soak so that clock samples see the GPU under this load
-    soak_end = time.time() + args.soak
-    while time.time() < soak_end:
-        with torch.cuda.stream(stream):
-            graph.replay()
-        stream.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):            # replay() launches on the current stream
-        ev0.record(stream)
-        for _ in range(reps):
-            graph.replay()
-        ev1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(ms, world)
-    ms_per_step = ms / steps_run
-    value = aggregate_gbs(world, bytes_per_step, steps_run, ms)
-
-    # dominant kernel alone: the library brackets each kernel with events on the
-    # launching stream; a GPU-side sleep queued first lets every profiled launch
-    # queue up behind it, so the kernels run back to back with no host gaps
-    S.sdpa_profile_enable(True)
-    S.sdpa_profile_collect()
-    with torch.cuda.stream(stream):
-        torch.cuda._sleep(20_000_000)          # ~10 ms of GPU time while the host enqueues
-        for r in range(2 * copies):
-            call(S, c, t, ks[r % copies], vs[r % copies], out, sp)
-    torch.cuda.synchronize()
-    prof = S.sdpa_profile_collect()
-    S.sdpa_profile_enable(False)
-    n_dec, ms_dec = prof["decode_mma"]
-    n_cmb, ms_cmb = prof["combine"]
-    dec_us_isolated = 1e3 * ms_dec / max(n_dec, 1)
-    # The decode kernel is the only kernel of a step (launches_per_step == 1 on
-    # this path): its average launch duration over the timed region is the
-    # timed region's duration divided by the launches in it.
+    r = time_decode(S, w, rank, world, stream, steps, warmup, args.soak, ClockSampler(local))
+    ms_per_step = r["ms"] / steps
+    value = aggregate_gbs(world, bytes_per_step, steps, r["ms"])
+    launches_per_step = r["launches"]
+    # The decode kernel is the only kernel of a step (one launch per call on this
+    # path): its average launch duration over the timed region is the timed
+    # region's duration divided by the launches in it.
     dec_us = 1e3 * ms_per_step / max(launches_per_step, 1)
     achieved = bytes_per_step / (dec_us * 1e-6) / 1e9
     traffic = ncu_traffic(f"decode_mma kL={args.kl}", ["decode_mma.cu", "common.cuh", "kernels.h"])
@@ -325,36 +366,71 @@ def run_ours(args, peaks):
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
             "traffic": traffic, "algorithmic_bytes_per_launch": bytes_per_step,
             "kernel_us": round(dec_us, 3), "launches_per_step": launches_per_step,
-            "kernel_us_isolated": round(dec_us_isolated, 3),
-            "combine_us": round(1e3 * ms_cmb / max(n_cmb, 1), 3),
-            "timing": "kernel_us = timed region / launches in it (CUDA events on the launching stream); "
-                      "kernel_us_isolated = event pair around each eager launch",
+            "kernel_us_isolated": round(r["us_isolated"], 3),
+            "frac_isolated": round(bytes_per_step / (r["us_isolated"] * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+            "timing": "kernel_us = timed region / launches in it (CUDA events on the launching stream, "
+                      "graph replay, consecutive launches overlap their prologues); kernel_us_isolated = "
+                      "event pair around each launch, launches queued back to back",
             "peak_source": f"{peaks['source']} hbm_gbs (copy, burst)"}
 
-    result = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": steps_run,
-              "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
+    result = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": steps,
+              "warmup": warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
               "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-              "config": {"workload": w["name"], "kv_copies_rotated": copies,
-                         "l2": f"inputs larger than L2: {copies} rotating K/V copies "
-                               f"({copies * kv_bytes / 2**20:.0f} MiB > 126 MB L2)",
-                         "launch": "CUDA graph replay of the C-ABI calls", "soak_s": args.soak,
+              "config": {"workload": w["name"], "kv_copies_rotated": r["copies"],
+                         "l2": f"inputs larger than L2: {r['copies']} rotating K/V copies "
+                               f"({r['copies'] * r['kv_bytes'] / 2**20:.0f} MiB > 126 MB L2)",
+                         "launch": "CUDA graph of the C-ABI calls, one replay", "soak_s": args.soak,
                          "parallelism": f"replicas x{world} (no collective)"},
-               "roofline": roof, "clocks": clk, "gpu_launches": launches_per_step * steps_run}
+              "roofline": roof, "clocks": r["clocks"], "gpu_launches": launches_per_step * steps}
 
     if not args.no_e2e:
+        c, t = device_case(w, rank)
+        out = torch.empty(c.B * c.Hq * c.Lq * c.Dv, dtype=t["q"].dtype, device="cuda")
         result["e2e"] = e2e(S, c, t, out, stream, args, world)
+        del c, t, out
+    if not args.no_extra:
+        result["decode"] = decode_leg(S, stream, peaks, rank, world, args)
     if not args.no_prefill:
         result["prefill"] = prefill_leg(S, stream, peaks, rank, args, local)
-    if not args.no_prefill:
         result["mla_decode"] = mla_leg(S, stream, peaks, rank, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        if not args.no_extra:
+            result["cpu_baseline_configs"] = cpu_baseline_configs(args.cpu_seconds / 4)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
         import torch.distributed as dist
-        del graph
         dist.destroy_process_group()
+
+
+DECODE_EXTRA = [
+    decode_workload(1024),
+    dict(name="decode bf16 B=1 qL=1 kL=4096 Hq=32 Hkv=16 D=256 sliding window 1024 (Gemma-4 sliding-layer shape)",
+         seed=1011, B=1, Hq=32, Hkv=16, Lq=1, Lk=4096, Dqk=256, Dv=256, dtype="bf16", mask="sliding", window=1024,
+         layout="bhld"),
+    dict(name="decode bf16 B=1 qL=1 kL=1024 Hq=32 Hkv=4 D=512 no mask", seed=1002, B=1, Hq=32, Hkv=4, Lq=1,
+         Lk=1024, Dqk=512, Dv=512, dtype="bf16", mask="none", layout="bhld"),
+    dict(name="decode bf16 B=1 qL=1 kL=4096 Hq=32 Hkv=4 D=512 no mask", seed=1002, B=1, Hq=32, Hkv=4, Lq=1,
+         Lk=4096, Dqk=512, Dv=512, dtype="bf16", mask="none", layout="bhld"),
+]
+
+
+def decode_leg(S, stream, peaks, rank, world, args):
+    """The other decode configurations, timed like the headline (graph replay of
+    exactly --steps calls over rotating K/V copies larger than L2)."""
+    res = []
+    for w in DECODE_EXTRA:
+        r = time_decode(S, w, rank, world, stream, args.steps, max(args.warmup, 3), 0.2)
+        nb = decode_bytes(w)
+        us = 1e3 * r["ms"] / args.steps / max(r["launches"], 1)
+        gbs = nb / (us * 1e-6) / 1e9
+        res.append({"workload": w["name"], "us_per_call": round(us, 3),
+                    "us_isolated": round(r["us_isolated"], 3), "algorithmic_bytes": nb,
+                    "achieved_gbs": round(gbs, 1), "peak_gbs": peaks["hbm_gbs"],
+                    "frac": round(gbs / peaks["hbm_gbs"], 4), "bound": "hbm", "launches_per_call": r["launches"],
+                    "steps": args.steps, "kv_copies_rotated": r["copies"]})
+    return res
 
 
 def run_prefill_only(args, peaks):
@@ -484,7 +560,8 @@ def prefill_leg(S, stream, peaks, rank, args, local=0):
         sp = stream.cuda_stream
         clocks = ClockSampler(local) if args.prefill_soak > 0 else None
         with torch.cuda.stream(stream):
-            call(S, c, t, t["k"], t["v"], out, sp)
+            for _ in range(10):                 # warm-up launches
+                call(S, c, t, t["k"], t["v"], out, sp)
             torch.cuda.synchronize()
             if clocks:
                 clocks.start()
@@ -502,19 +579,29 @@ def prefill_leg(S, stream, peaks, rank, args, local=0):
                 e1.record(stream)
         torch.cuda.synchronize()
         clk = clocks.stop() if clocks else None
-        ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / n
+        times = [e0.elapsed_time(e1) for e0, e1 in evs]
+        ms = statistics.median(times)
         fl = prefill_flops(w)
         tf = fl / (ms * 1e-3) / 1e12
         cnt = S.sdpa_get_counters()
-        fp32 = w["dtype"] == "f32"
-        peak = FFMA_TFLOPS if fp32 else peaks["bf16_tflops"]
-        entry = {"workload": w["name"], "ms": round(ms, 4), "tflops": round(tf, 2),
-                 "algorithmic_flops": fl, "peak_tflops": round(peak, 1),
-                 "peak_source": "FFMA: 148 SMs x 128 lanes x 2 x 1.965 GHz (nominal)" if fp32
-                 else f"{peaks['source']} bf16_tflops (cuBLAS, burst)",
-                 "frac": round(tf / peak, 4), "bound": "alu" if fp32 else "tensor",
-                 "kernel": "prefill_tcgen05" if cnt["prefill_tcgen05_launches"] else "prefill_ffma",
-                 "iters": n, "l2": "flushed between timed launches"}
+        kernel = ("prefill_tcgen05" if cnt["prefill_tcgen05_launches"] else
+                  "prefill_tf32x3" if cnt["prefill_tf32_launches"] else "prefill_ffma")
+        if kernel == "prefill_ffma":
+            peak, src, bound = FFMA_TFLOPS, "FFMA: 148 SMs x 128 lanes x 2 x 1.965 GHz (nominal)", "alu"
+        elif kernel == "prefill_tf32x3":
+            peak = peaks["bf16_tflops"] * TF32_OVER_BF16
+            src = (f"{peaks['source']} bf16_tflops x 1.1/2.25 (nominal dense tf32/bf16); "
+                   "3 tf32 MMAs per product, so frac <= 1/3 and tensor_pipe_frac = 3 x frac")
+            bound = "tensor"
+        else:
+            peak, src, bound = peaks["bf16_tflops"], f"{peaks['source']} bf16_tflops (cuBLAS, burst)", "tensor"
+        entry = {"workload": w["name"], "ms": round(ms, 4), "ms_min": round(min(times), 4),
+                 "ms_max": round(max(times), 4), "tflops": round(tf, 2),
+                 "algorithmic_flops": fl, "peak_tflops": round(peak, 1), "peak_source": src,
+                 "frac": round(tf / peak, 4), "bound": bound, "kernel": kernel,
+                 **({"tensor_pipe_frac": round(3 * tf / peak, 4)} if kernel == "prefill_tf32x3" else {}),
+                 "iters": n, "warmup": 10, "timing": "median of the timed launches",
+                 "l2": "flushed between timed launches"}
         if clk:
             entry["clocks"] = clk
         res.append(entry)
@@ -558,7 +645,7 @@ def mla_leg(S, stream, peaks, rank, args):
                 call(S, c, t, t["k"], t["v"], out, sp)
                 e1.record(stream)
         torch.cuda.synchronize()
-        us = 1e3 * sum(e0.elapsed_time(e1) for e0, e1 in evs) / n
+        us = 1e3 * statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
         e = 4 if dt == "f32" else 2
         nbytes = e * (c.B * c.Hkv * c.Lk * c.Dqk + c.B * c.Hq * c.Lq * (c.Dqk + c.Dv))
         gbs = nbytes / (us * 1e-6) / 1e9
@@ -566,7 +653,7 @@ def mla_leg(S, stream, peaks, rank, args):
                     "algorithmic_bytes": nbytes, "mask_bytes": e * c.Lk, "achieved_gbs": round(gbs, 1),
                     "peak_gbs": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4),
                     "bound": "latency (0.3-0.7 MB per call: memory round trips and two launches, not bandwidth)", "launches_per_call": S.sdpa_last_launch_count(),
-                    "iters": n, "l2": "flushed between timed launches"})
+                    "iters": n, "timing": "median", "l2": "flushed between timed launches"})
         del t, out
     del flush
     return res
@@ -592,6 +679,63 @@ def cpu_baseline(w, seconds):
     return {"value": round(decode_bytes(w) * n / el / 1e9, 4), "unit": "GB/s", "cores": min(threads, c.B * c.Hq),
             "kind": "oracle", "sample": f"{n} full decode steps ({c.B * c.Hq} query rows x {c.Lk} keys each) "
                                         f"in {el:.1f} s; rows split over host threads"}
+
+
+ORACLE_CONFIGS = [
+    dict(name="config 1: fp32 B=2 L=82 H=8 D=64 no mask [B,L,H,D] (N(0,1) copy)", seed=1000, B=2, Hq=8, Hkv=8,
+         Lq=82, Lk=82, Dqk=64, Dv=64, dtype="f32", mask="none", layout="blhd", kind="prefill"),
+    dict(decode_workload(1024), kind="decode"),
+    dict(DECODE_EXTRA[2], kind="decode"),
+    dict(DECODE_EXTRA[3], kind="decode"),
+    dict(PREFILL_WORKLOADS[3], kind="prefill"),
+    dict(PREFILL_WORKLOADS[0], kind="prefill"),
+    dict(PREFILL_WORKLOADS[1], kind="prefill"),
+    dict(PREFILL_WORKLOADS[2], kind="prefill"),
+]
+
+
+def cpu_baseline_configs(seconds):
+    """The float64 oracle, as it stands, on configs 1-4 (host cores, rows split
+    over threads).  Decode configs and config 1 run whole calls; the large
+    prefill configs run seeded samples of query rows for about `seconds` each,
+    and their throughput is extrapolated from the time per row."""
+    import oracle
+    from scaled_dot_product_14_b200 import inputs as I
+    oracle.build()
+    threads = usable_cpus()
+    res = []
+    for w in ORACLE_CONFIGS:
+        c = I.make_case(w["seed"], w["B"], w["Hq"], w["Hkv"], w["Lq"], w["Lk"], w["Dqk"], w["Dv"],
+                        dtype=I.DTYPE_BY_NAME[w["dtype"]], mask=w["mask"], layout=w["layout"])
+        total_rows = c.B * c.Hq * c.Lq
+        args = dict(B=c.B, Hq=c.Hq, Hkv=c.Hkv, Lq=c.Lq, Lk=c.Lk, Dqk=c.Dqk, Dv=c.Dv, strides=c.strides,
+                    scale=c.scale, dtype=c.dtype, mask_kind=c.mask_kind, mask=c.mask, mask_strides=c.mask_strides,
+                    threads=threads)
+        whole = total_rows * c.Lk <= 2 ** 22
+        n_rows, t0, calls = 0, time.time(), 0
+        while True:
+            if whole:
+                oracle.sdpa_rows(c.q, c.k, c.v, **args)
+                n_rows += total_rows
+            else:
+                rows = I.sample_rows(w["seed"] + calls, c.B, c.Hq, c.Lq, 4 * threads, include_edges=False)
+                oracle.sdpa_rows(c.q, c.k, c.v, rows=rows, **args)
+                n_rows += len(rows)
+            calls += 1
+            if time.time() - t0 >= seconds:
+                break
+        el = time.time() - t0
+        est_s = el / n_rows * total_rows          # one whole call
+        if w["kind"] == "decode":
+            val, unit = decode_bytes(w) / est_s / 1e9, "GB/s"
+        else:
+            val, unit = prefill_flops(w) / est_s / 1e12, "TFLOP/s"
+        res.append({"workload": w["name"], "value": round(val, 6), "unit": unit, "cores": threads,
+                    "kind": "oracle", "seconds_per_call": round(est_s, 4),
+                    "sample": (f"{calls} whole calls in {el:.1f} s" if whole else
+                               f"{n_rows} seeded query rows of {total_rows} in {el:.1f} s; "
+                               f"extrapolated per row x rows")})
+    return res
 
 
 # ----------------------------------------------------------------------------- reference arm (the oracle)
@@ -646,7 +790,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the prefill workloads and print their lines (profiling)")
-    ap.add_argument("--prefill-iters", type=int, default=20)
+    ap.add_argument("--prefill-iters", type=int, default=50)
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other decode configurations and the oracle timing on configs 1-4")
     ap.add_argument("--prefill-soak", type=float, default=1.0,
                     help="untimed seconds per prefill workload while clocks are sampled (0: no sampling)")
     args = ap.parse_args()

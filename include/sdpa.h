@@ -22,7 +22,9 @@
  *     issue #1065, section "Why this is a precision problem" (keys = 32 latent
  *     + 8 rope columns, values = the 32 latent columns, so v may point at k
  *     with k's strides); these dims run on the CUDA-core kernels;
- *   - masks: none, additive, boolean, causal (MLX PR #4330, "Proposed changes").
+ *   - masks: none, additive, boolean, causal (MLX PR #4330, "Proposed changes"),
+ *     and a causal sliding window (the local-attention layers of Gemma 4's
+ *     hybrid layout, MLX issue #3885, "Current routing"; sdpa_forward_window).
  *
  * Layout is never inferred from a tensor's shape: every tensor is passed as a
  * base pointer plus explicit (b, h, l, d) element strides, so [B,L,H,D] and
@@ -35,6 +37,8 @@
  *   - boolean mask: nonzero = attend, zero = removed;
  *   - causal with Lq != Lk is aligned bottom-right: key j is visible to query
  *     i iff j <= i + (Lk - Lq);
+ *   - sliding window of W keys, with the same alignment: key j is visible to
+ *     query i iff i + (Lk - Lq) - W < j <= i + (Lk - Lq);
  *   - a query row with no visible key yields zeros (never NaN).
  *
  * Threading: the functions are thread-safe.  Execution is asynchronous on the
@@ -59,7 +63,8 @@ extern "C" {
 
 /* Element types of q, k, v, out (and of an additive mask). */
 typedef enum {
-    SDPA_F32 = 0,   /* IEEE binary32; computed in true fp32 (no TF32, no fp16 rounding) */
+    SDPA_F32 = 0,   /* IEEE binary32; fp32-class accuracy: FFMA, or TF32 tensor cores only with
+                       the three-term split hi*hi + hi*lo + lo*hi (never plain TF32 or fp16) */
     SDPA_F16 = 1,   /* IEEE binary16 storage, fp32 accumulation */
     SDPA_BF16 = 2   /* bfloat16 storage, fp32 accumulation */
 } sdpa_dtype;
@@ -68,7 +73,9 @@ typedef enum {
     SDPA_MASK_NONE = 0,      /* mask must be NULL */
     SDPA_MASK_ADDITIVE = 1,  /* mask: same element type as q, added to scale*q.k */
     SDPA_MASK_BOOL = 2,      /* mask: uint8, nonzero = attend */
-    SDPA_MASK_CAUSAL = 3     /* mask must be NULL; bottom-right aligned */
+    SDPA_MASK_CAUSAL = 3,    /* mask must be NULL; bottom-right aligned */
+    SDPA_MASK_SLIDING = 4    /* causal sliding window; only through sdpa_forward_window (which
+                                carries the window length); sdpa_supported accepts it */
 } sdpa_mask_kind;
 
 typedef enum {
@@ -90,7 +97,9 @@ typedef enum {
 
 typedef enum {
     SDPA_PATH_NONE = 0,     /* empty problem: nothing to launch */
-    SDPA_PATH_PREFILL = 1,  /* Lq > 8: tiled flash kernel (tcgen05 for fp16/bf16, FFMA for fp32) */
+    SDPA_PATH_PREFILL = 1,  /* Lq > 8: tiled flash kernel (tcgen05 kind::f16 for fp16/bf16; for fp32
+                               tcgen05 kind::tf32 with a three-term hi/lo split at head dims
+                               (40,32), 64, 72, 80, 96, FFMA at the others) */
     SDPA_PATH_DECODE = 2    /* Lq <= 8: split-K kernel plus log-sum-exp combine */
 } sdpa_path;
 
@@ -112,6 +121,7 @@ typedef enum {
  *                  element type = dtype; strides in elements, 0 broadcasts.
  *        BOOL:     same indexing, uint8 elements.
  *        NONE / CAUSAL: mask and mask_strides must be NULL.
+ *        SLIDING: refused here (SDPA_ERR_INVALID_ARG); use sdpa_forward_window.
  * dtype : sdpa_dtype of q, k, v, out.
  * stream: a cudaStream_t (NULL = the legacy default stream).
  *
@@ -122,7 +132,10 @@ typedef enum {
  * Ownership: all pointers are the caller's.  The decode path uses a split-K
  * workspace the library allocates on first use per (device, stream), keeps,
  * and frees in sdpa_shutdown(); two calls on the same stream share it safely
- * because the stream orders them.
+ * because the stream orders them.  A larger problem grows the workspace
+ * without freeing the smaller buffer (a CUDA graph captured earlier may still
+ * use it), so graphs captured with sdpa_forward calls stay valid until
+ * sdpa_shutdown.
  * Returns an sdpa_status.  On any status other than SDPA_OK and SDPA_ERR_CUDA
  * nothing was launched.
  */
@@ -133,6 +146,25 @@ int sdpa_forward(const void* q, const void* k, const void* v, void* out,
                  int dtype, void* stream);
 
 /*
+ * sdpa_forward_window -- causal sliding-window (local) attention: with
+ * own = i + (Lk - Lq), key j is visible to query i iff own - window < j <= own,
+ * the `window` most recent keys up to the query's own bottom-right-aligned
+ * position.  Gemma 4's hybrid layout interleaves such layers with global ones
+ * (MLX issue #3885, "Current routing"); the pages give no rule for the
+ * window, and this is the plainest reading of local causal attention.
+ * window >= Lk is plain causal attention; a query whose window holds no key
+ * (own < 0) yields zeros.
+ *
+ * Arguments are those of sdpa_forward without the mask arguments; window >= 1
+ * (else SDPA_ERR_INVALID_ARG).  Both paths skip every key tile that lies
+ * outside all of a CTA's windows: those keys are never loaded.
+ */
+int sdpa_forward_window(const void* q, const void* k, const void* v, void* out,
+                        int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk,
+                        int64_t Dqk, int64_t Dv, const int64_t strides[16], float scale,
+                        int64_t window, int dtype, void* stream);
+
+/*
  * sdpa_forward_noalloc -- sdpa_forward for callers that cannot allocate device
  * memory when they call attention: a process whose memory manager already owns
  * the whole GPU (a caching allocator, a serving runtime with a fixed memory
@@ -141,8 +173,10 @@ int sdpa_forward(const void* q, const void* k, const void* v, void* out,
  * no counterpart of this entry point.
  *
  * Arguments, layout, validation and result are those of sdpa_forward, but it
- * covers only the decode path with fp16 / bf16 (Lq <= 8); other problems return
- * SDPA_ERR_INVALID_ARG (an empty problem returns SDPA_OK).  It allocates
+ * covers only the decode path with fp16 / bf16 (Lq <= 8) on the head dims of
+ * the tensor-core decode kernel (every supported pair except the absorbed-MLA
+ * (40, 32)); other problems return SDPA_ERR_INVALID_ARG, decided before any
+ * CUDA call (an empty problem returns SDPA_OK).  It allocates
  * nothing: the split-K partials and the per-group completion counters go to
  * a 4 MiB array compiled into the library (the counters take its first 64 KiB
  * and are cleared by each call with a memset on `stream`), which every GPU
@@ -194,6 +228,7 @@ typedef struct {
     uint64_t decode_mma_launches;       /* fp16/bf16 split-K decode */
     uint64_t decode_ffma_launches;      /* fp32 split-K decode */
     uint64_t combine_launches;          /* log-sum-exp combine of split-K partials */
+    uint64_t prefill_tf32_launches;     /* fp32 prefill on tcgen05 kind::tf32, three-term split */
 } sdpa_counters;
 
 void sdpa_get_counters(sdpa_counters* out);
@@ -208,9 +243,43 @@ int sdpa_last_launch_count(void);
 /*
  * Reads and clears the device-side error flag that bounded in-kernel waits
  * set when they give up (0 = none).  Synchronises the stream.  Returns an
- * sdpa_status: SDPA_ERR_TIMEOUT if the flag was set.
+ * sdpa_status: SDPA_ERR_TIMEOUT if the flag was set; in that case it also
+ * zeroes the decode split-barrier counters of this (device, stream)'s
+ * workspace (on the stream, synchronously), so the next decode call on the
+ * stream starts from a clean barrier whatever the timed-out call left.
  */
 int sdpa_check_device_error(void* stream, int* code_out);
+
+/*
+ * Test and diagnostic hooks; none is needed in normal use.  Each is
+ * process-wide and applies from the next call.  They exist so that the
+ * failure paths (a bounded wait that runs out, a workspace that cannot be
+ * allocated) can be exercised without faulting or hanging a GPU.
+ *   SDPA_DEBUG_WAIT_LIMIT_NS: every bounded wait of the fp16/bf16 decode
+ *       kernel gives up after `value` nanoseconds instead of about 2 s
+ *       (value <= 0 restores the default).
+ *   SDPA_DEBUG_DECODE_BARRIER_EXTRA: added to the number of split arrivals
+ *       the decode kernel's split barrier waits for (0..1024; 0 restores).
+ *       A value > 0 makes the target unreachable: every CTA's wait runs out
+ *       after the wait limit, the device error flag is set (read it with
+ *       sdpa_check_device_error) and the output is left unwritten.
+ *   SDPA_DEBUG_FAIL_ALLOCS: the next `value` calls of sdpa_forward that need
+ *       split-K workspace fail as if the allocation had failed: they return
+ *       SDPA_ERR_NO_MEMORY and launch nothing.
+ * Returns SDPA_OK, or SDPA_ERR_INVALID_ARG for an unknown knob or a value out
+ * of range.
+ */
+typedef enum {
+    SDPA_DEBUG_WAIT_LIMIT_NS = 0,
+    SDPA_DEBUG_DECODE_BARRIER_EXTRA = 1,
+    SDPA_DEBUG_FAIL_ALLOCS = 2
+} sdpa_debug_knob;
+
+int sdpa_debug_set(int knob, int64_t value);
+
+/* Bytes of split-K workspace sdpa_forward currently holds, over every device
+ * and stream (0 before the first decode call that splits keys). */
+int64_t sdpa_workspace_bytes(void);
 
 /*
  * Optional per-kernel timing with CUDA events (off by default).  While
@@ -227,7 +296,8 @@ typedef enum {
     SDPA_KERNEL_DECODE_FFMA = 3,
     SDPA_KERNEL_COMBINE = 4,
     SDPA_KERNEL_ZERO_FILL = 5,
-    SDPA_KERNEL_FAMILIES = 6
+    SDPA_KERNEL_PREFILL_TF32 = 6,
+    SDPA_KERNEL_FAMILIES = 7
 } sdpa_kernel_family;
 
 int sdpa_profile_enable(int on);
@@ -236,7 +306,8 @@ int sdpa_profile_collect(uint64_t launches[SDPA_KERNEL_FAMILIES], double total_m
 /* Frees every cached workspace.  Call with no sdpa work in flight. */
 int sdpa_shutdown(void);
 
-/* ABI version of this header (increases on incompatible change). */
+/* ABI version of this header (increases on incompatible change): 2 added the
+ * sliding-window entry point, the tf32 counter and kernel family. */
 int sdpa_abi_version(void);
 
 #ifdef __cplusplus

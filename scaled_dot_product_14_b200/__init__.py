@@ -22,7 +22,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "sdpa.h")
 
 # sdpa_dtype / sdpa_mask_kind / sdpa_path / sdpa_status (include/sdpa.h)
 SDPA_F32, SDPA_F16, SDPA_BF16 = 0, 1, 2
-SDPA_MASK_NONE, SDPA_MASK_ADDITIVE, SDPA_MASK_BOOL, SDPA_MASK_CAUSAL = 0, 1, 2, 3
+SDPA_MASK_NONE, SDPA_MASK_ADDITIVE, SDPA_MASK_BOOL, SDPA_MASK_CAUSAL, SDPA_MASK_SLIDING = 0, 1, 2, 3, 4
 SDPA_PATH_NONE, SDPA_PATH_PREFILL, SDPA_PATH_DECODE = 0, 1, 2
 STATUS = {0: "SDPA_OK", 1: "SDPA_ERR_INVALID_ARG", 2: "SDPA_ERR_UNSUPPORTED_DIM", 3: "SDPA_ERR_UNSUPPORTED_STRIDE",
           4: "SDPA_ERR_MISALIGNED", 5: "SDPA_ERR_LAUNCH_CONFIG", 6: "SDPA_ERR_CUDA", 7: "SDPA_ERR_TIMEOUT",
@@ -41,7 +41,8 @@ class SdpaError(RuntimeError):
 class _Counters(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in (
         "calls", "prefill_calls", "decode_calls", "empty_calls", "rejected_calls", "prefill_tcgen05_launches",
-        "prefill_ffma_launches", "decode_mma_launches", "decode_ffma_launches", "combine_launches")]
+        "prefill_ffma_launches", "decode_mma_launches", "decode_ffma_launches", "combine_launches",
+        "prefill_tf32_launches")]
 
 
 _lib = None
@@ -64,6 +65,9 @@ def lib() -> ctypes.CDLL:
                                        vp, P64, i32, vp]
             L.sdpa_forward_noalloc.restype = i32
             L.sdpa_forward_noalloc.argtypes = list(L.sdpa_forward.argtypes)
+            L.sdpa_forward_window.restype = i32
+            L.sdpa_forward_window.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, P64,
+                                              ctypes.c_float, i64, i32, vp]
             L.sdpa_supported.restype = i32
             L.sdpa_supported.argtypes = [i64, i64, i64, i64, i64, i64, i64, P64, i32, P64, i32,
                                          ctypes.POINTER(ctypes.c_int)]
@@ -82,6 +86,10 @@ def lib() -> ctypes.CDLL:
             L.sdpa_profile_enable.argtypes = [i32]
             L.sdpa_profile_collect.restype = i32
             L.sdpa_profile_collect.argtypes = [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_double)]
+            L.sdpa_debug_set.restype = i32
+            L.sdpa_debug_set.argtypes = [i32, i64]
+            L.sdpa_workspace_bytes.restype = i64
+            L.sdpa_workspace_bytes.argtypes = []
             _lib = L
     return _lib
 
@@ -101,6 +109,12 @@ def sdpa_forward(q, k, v, out, B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, scale, mask
     """Calls the C entry point; pointers are ints (device addresses), strides sequences."""
     return lib().sdpa_forward(q, k, v, out, B, Hq, Hkv, Lq, Lk, Dqk, Dv, _i64array(strides, 16),
                               ctypes.c_float(scale), mask_kind, mask, _i64array(mask_strides, 4), dtype, stream)
+
+
+def sdpa_forward_window(q, k, v, out, B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, scale, window, dtype, stream) -> int:
+    """Causal sliding-window attention over the `window` most recent keys."""
+    return lib().sdpa_forward_window(q, k, v, out, B, Hq, Hkv, Lq, Lk, Dqk, Dv, _i64array(strides, 16),
+                                     ctypes.c_float(scale), int(window), dtype, stream)
 
 
 def sdpa_forward_noalloc(q, k, v, out, B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, scale, mask_kind, mask,
@@ -155,7 +169,20 @@ def sdpa_abi_version() -> int:
     return lib().sdpa_abi_version()
 
 
-KERNEL_FAMILIES = ("prefill_tcgen05", "prefill_ffma", "decode_mma", "decode_ffma", "combine", "zero_fill")
+# sdpa_debug_knob (include/sdpa.h): test hooks for the failure paths
+SDPA_DEBUG_WAIT_LIMIT_NS, SDPA_DEBUG_DECODE_BARRIER_EXTRA, SDPA_DEBUG_FAIL_ALLOCS = 0, 1, 2
+
+
+def sdpa_debug_set(knob: int, value: int) -> int:
+    return lib().sdpa_debug_set(knob, int(value))
+
+
+def sdpa_workspace_bytes() -> int:
+    return lib().sdpa_workspace_bytes()
+
+
+KERNEL_FAMILIES = ("prefill_tcgen05", "prefill_ffma", "decode_mma", "decode_ffma", "combine", "zero_fill",
+                   "prefill_tf32")
 
 
 def sdpa_profile_enable(on: bool) -> int:
@@ -182,13 +209,14 @@ def _dtype_code(t):
     return codes[t.dtype]
 
 
-def attention(q, k, v, *, scale=None, mask=None, causal=False, out=None, stream=None):
+def attention(q, k, v, *, scale=None, mask=None, causal=False, window=None, out=None, stream=None):
     """out = softmax(scale q k^T + mask) v for CUDA tensors given as logical [B, H, L, D] views.
 
     ``mask``: None; a bool tensor (True = attend) or a tensor of q's dtype
     (additive), 4-D and broadcastable to [B, Hq, Lq, Lk] through zero strides
-    (``expand``).  ``causal=True`` uses bottom-right alignment.  Returns ``out``
-    ([B, Hq, Lq, Dv], contiguous unless given).
+    (``expand``).  ``causal=True`` uses bottom-right alignment; with ``window``
+    it is limited to the ``window`` most recent keys (sliding window).
+    Returns ``out`` ([B, Hq, Lq, Dv], contiguous unless given).
     """
     import torch
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
@@ -219,6 +247,14 @@ def attention(q, k, v, *, scale=None, mask=None, causal=False, out=None, stream=
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     strides = list(q.stride()) + list(k.stride()) + list(v.stride()) + list(out.stride())
+    if window is not None:
+        if not causal:
+            raise ValueError("a sliding window is causal: pass causal=True with window")
+        st = sdpa_forward_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, Lq, Lk,
+                                 Dqk, Dv, strides, float(scale), int(window), dt, stream)
+        if st != 0:
+            raise SdpaError(st, "sdpa_forward_window")
+        return out
     st = sdpa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, Lq, Lk, Dqk, Dv,
                       strides, float(scale), mk, mptr, mst, dt, stream)
     if st != 0:

@@ -40,10 +40,15 @@ namespace sdpa {
 namespace {
 
 std::atomic<uint64_t> c_calls{0}, c_prefill{0}, c_decode{0}, c_empty{0}, c_rejected{0};
-std::atomic<uint64_t> c_tc{0}, c_pffma{0}, c_dmma{0}, c_dffma{0}, c_combine{0};
+std::atomic<uint64_t> c_tc{0}, c_pffma{0}, c_dmma{0}, c_dffma{0}, c_combine{0}, c_tf32{0};
 
 thread_local std::string t_last_cuda_error;
 thread_local int t_last_launches = 0;
+
+// test hooks (sdpa_debug_set)
+std::atomic<int64_t> g_dbg_wait_limit_ns{0};    // <= 0: the default limit
+std::atomic<int64_t> g_dbg_barrier_extra{0};
+std::atomic<int64_t> g_dbg_fail_allocs{0};
 
 bool env_flag(const char* name) {
     const char* v = getenv(name);
@@ -82,7 +87,7 @@ int validate(int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk, int64_t
              const int64_t* strides, int mask_kind, const int64_t* mask_strides, int dtype, int* path) {
     *path = SDPA_PATH_NONE;
     if (dtype < SDPA_F32 || dtype > SDPA_BF16) return SDPA_ERR_INVALID_ARG;
-    if (mask_kind < SDPA_MASK_NONE || mask_kind > SDPA_MASK_CAUSAL) return SDPA_ERR_INVALID_ARG;
+    if (mask_kind < SDPA_MASK_NONE || mask_kind > SDPA_MASK_SLIDING) return SDPA_ERR_INVALID_ARG;
     if (B < 0 || Hq < 0 || Hkv <= 0 || Lq < 0 || Lk < 0) return SDPA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return SDPA_ERR_INVALID_ARG;
     if (!dims_supported(Dqk, Dv)) return SDPA_ERR_UNSUPPORTED_DIM;
@@ -134,51 +139,64 @@ int device_info(DeviceInfo* out) {
 }
 
 // ---------------------------------------------------------------- split-K workspace
-// Per (device, stream): split-K partials (contents do not outlive a call) and
-// the decode kernel's per-group counters (zero between calls: zeroed when
-// allocated, and every call leaves them zero).
+// Per (device, stream): the split-K partials (contents do not outlive a call)
+// and the decode kernel's arrival counters.  A grown partial buffer does not
+// free the smaller one (a CUDA graph captured earlier may still point at it):
+// retired buffers are kept until sdpa_shutdown.  The counters come in one
+// zero-initialised region per launch shape (groups, splits): every call of a
+// shape adds exactly its split count to each of its groups' counters, which is
+// what the kernel's barrier relies on, so shapes never share counters.
 struct Workspace {
     void* ptr = nullptr;
     size_t bytes = 0;
-    int* counters = nullptr;
-    size_t n_counters = 0;
+    std::vector<std::pair<void*, size_t>> retired;
+    std::map<std::tuple<int64_t, int, int>, std::pair<int*, size_t>> counters;
 };
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
-int workspace(int dev, cudaStream_t stream, size_t bytes, size_t n_counters, void** out, int** counters) {
+int workspace(int dev, cudaStream_t stream, size_t bytes, void** out) {
     std::lock_guard<std::mutex> lk(g_mu);
+    // test hook: behave as if the allocator had no memory, before touching anything
+    for (int64_t n = g_dbg_fail_allocs.load(); n > 0;)
+        if (g_dbg_fail_allocs.compare_exchange_weak(n, n - 1)) {
+            t_last_cuda_error = "workspace allocation failed (forced by SDPA_DEBUG_FAIL_ALLOCS)";
+            return SDPA_ERR_NO_MEMORY;
+        }
     Workspace& w = g_ws[{dev, stream}];
     if (w.bytes < bytes) {
-        if (w.ptr) cudaFreeAsync(w.ptr, stream);
-        w.ptr = nullptr;
-        w.bytes = 0;
-        size_t want = bytes + bytes / 4 + 4096;
-        cudaError_t e = cudaMallocAsync(&w.ptr, want, stream);
+        const size_t want = bytes + bytes / 4 + 4096;
+        void* ptr = nullptr;
+        cudaError_t e = cudaMallocAsync(&ptr, want, stream);
         if (e != cudaSuccess) {
             cudaGetLastError();
-            w.ptr = nullptr;
             t_last_cuda_error = cudaGetErrorString(e);
             return SDPA_ERR_NO_MEMORY;
         }
+        if (w.ptr) w.retired.emplace_back(w.ptr, w.bytes);
+        w.ptr = ptr;
         w.bytes = want;
     }
-    if (w.n_counters < n_counters) {
-        if (w.counters) cudaFreeAsync(w.counters, stream);
-        w.counters = nullptr;
-        w.n_counters = 0;
-        const size_t want = n_counters + 1024;
-        cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&w.counters), want * sizeof(int), stream);
-        if (e == cudaSuccess) e = cudaMemsetAsync(w.counters, 0, want * sizeof(int), stream);
+    *out = w.ptr;
+    return SDPA_OK;
+}
+
+int counter_region(int dev, cudaStream_t stream, int64_t ctas, int lo, int extra, size_t n_ints, int** out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    Workspace& w = g_ws[{dev, stream}];
+    auto& slot = w.counters[std::make_tuple(ctas, lo, extra)];
+    if (slot.second < n_ints) {
+        int* c = nullptr;
+        cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&c), n_ints * sizeof(int), stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(c, 0, n_ints * sizeof(int), stream);
         if (e != cudaSuccess) {
             cudaGetLastError();
-            w.counters = nullptr;
             t_last_cuda_error = cudaGetErrorString(e);
             return SDPA_ERR_NO_MEMORY;
         }
-        w.n_counters = want;
+        if (slot.first) w.retired.emplace_back(slot.first, slot.second * sizeof(int));
+        slot = {c, n_ints};
     }
-    *out = w.ptr;
-    *counters = w.counters;
+    *out = slot.first;
     return SDPA_OK;
 }
 
@@ -207,6 +225,24 @@ int check_plan(const LaunchPlan& plan, const DeviceInfo& dev) {
 int cuda_fail(cudaError_t e) {
     t_last_cuda_error = cudaGetErrorString(e);
     return SDPA_ERR_CUDA;
+}
+
+// Zeroes the decode split-barrier counters of this (device, stream)'s
+// workspace, on that stream, and waits for it.
+int clear_counters(int dev, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_ws.find({dev, stream});
+    if (it == g_ws.end()) return SDPA_OK;
+    cudaError_t e = cudaSuccess;
+    for (auto& kv : it->second.counters)
+        if (e == cudaSuccess && kv.second.first)
+            e = cudaMemsetAsync(kv.second.first, 0, kv.second.second * sizeof(int), stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(e);
+    }
+    return SDPA_OK;
 }
 
 // ---------------------------------------------------------------- opt-in event timing
@@ -244,6 +280,12 @@ cudaError_t timed(int family, cudaStream_t stream, F&& fn) {
 }
 
 }  // namespace
+
+int record_cuda_error(cudaError_t e) {
+    cudaGetLastError();
+    return cuda_fail(e);
+}
+
 }  // namespace sdpa
 
 using namespace sdpa;
@@ -257,10 +299,15 @@ extern "C" int sdpa_supported(int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, in
     return st;
 }
 
-extern "C" int sdpa_forward(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t Hq,
-                            int64_t Hkv, int64_t Lq, int64_t Lk, int64_t Dqk, int64_t Dv,
-                            const int64_t strides[16], float scale, int mask_kind, const void* mask,
-                            const int64_t mask_strides[4], int dtype, void* stream_ptr) {
+namespace sdpa {
+namespace {
+
+// Both entry points: sdpa_forward (window = 0; the sliding kind is refused,
+// since it needs its window) and sdpa_forward_window (mask_kind = SLIDING).
+int forward_impl(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t Hq, int64_t Hkv,
+                 int64_t Lq, int64_t Lk, int64_t Dqk, int64_t Dv, const int64_t* strides, float scale,
+                 int mask_kind, const void* mask, const int64_t* mask_strides, int64_t window, int dtype,
+                 void* stream_ptr) {
     c_calls.fetch_add(1, std::memory_order_relaxed);
     t_last_launches = 0;
     auto reject = [](int st) {
@@ -270,6 +317,7 @@ extern "C" int sdpa_forward(const void* q, const void* k, const void* v, void* o
     int path = SDPA_PATH_NONE;
     int st = validate(B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, mask_kind, mask_strides, dtype, &path);
     if (st != SDPA_OK) return reject(st);
+    if ((mask_kind == SDPA_MASK_SLIDING) != (window > 0)) return reject(SDPA_ERR_INVALID_ARG);
     if (!std::isfinite(scale)) return reject(SDPA_ERR_INVALID_ARG);
     const bool needs_mask = (mask_kind == SDPA_MASK_ADDITIVE || mask_kind == SDPA_MASK_BOOL);
     if (needs_mask != (mask != nullptr)) return reject(SDPA_ERR_NULL_POINTER);
@@ -299,6 +347,12 @@ extern "C" int sdpa_forward(const void* q, const void* k, const void* v, void* o
     p.mask_kind = mask_kind;
     p.group = (int)(Hq / Hkv);
     p.splits = 1;
+    const int64_t lim = g_dbg_wait_limit_ns.load(std::memory_order_relaxed);
+    p.wait_limit_ns = lim > 0 ? (uint64_t)lim : kWaitLimitNs;
+    p.barrier_extra = (int)g_dbg_barrier_extra.load(std::memory_order_relaxed);
+    p.window = mask_kind == SDPA_MASK_SLIDING ? window : 0;
+    p.key_begin = 0;
+    if (mask_kind == SDPA_MASK_SLIDING && Lk - Lq - window + 1 > 0) p.key_begin = Lk - Lq - window + 1;
 
     const bool log = env_flag("SDPA_LOG");
     cudaError_t e;
@@ -323,9 +377,10 @@ extern "C" int sdpa_forward(const void* q, const void* k, const void* v, void* o
             const int64_t rows = B * Hq * Lq;
             const size_t o_bytes = (size_t)rows * p.splits * Dv * sizeof(float);
             const size_t l_bytes = (size_t)rows * p.splits * sizeof(float);
-            const size_t n_cnt = mma ? decode_mma_counters(p, plan) : 0;
             void* ws = nullptr;
-            if ((st = workspace(dev.device, stream, o_bytes + l_bytes + 256, n_cnt, &ws, &counters)) != SDPA_OK)
+            if ((st = workspace(dev.device, stream, o_bytes + l_bytes + 256, &ws)) != SDPA_OK) return reject(st);
+            if (mma && (st = counter_region(dev.device, stream, (int64_t)plan.grid.x, plan.split_lo,
+                                            plan.split_extra, decode_mma_counters(p, plan), &counters)) != SDPA_OK)
                 return reject(st);
             p.part_o = reinterpret_cast<float*>(ws);
             p.part_lse = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + ((o_bytes + 255) / 256) * 256);
@@ -346,17 +401,24 @@ extern "C" int sdpa_forward(const void* q, const void* k, const void* v, void* o
         }
         c_decode.fetch_add(1, std::memory_order_relaxed);
     } else {
+        // fp16 / bf16 on tcgen05 kind::f16; fp32 on tcgen05 kind::tf32 with the
+        // three-term split where its shared memory fits the head dims, else FFMA
         const bool tc = prefill_tc_supported(dtype, Dqk, Dv, p);
-        LaunchPlan plan = tc ? prefill_tc_plan(p, dtype, dev) : ffma_plan(p, dtype, dev, /*split_keys=*/false);
+        const bool tf = !tc && prefill_tf32_supported(dtype, Dqk, Dv);
+        LaunchPlan plan = tc   ? prefill_tc_plan(p, dtype, dev)
+                          : tf ? prefill_tf32_plan(p, dev)
+                               : ffma_plan(p, dtype, dev, /*split_keys=*/false);
         if ((st = check_plan(plan, dev)) != SDPA_OK) return reject(st);
         p.splits = plan.splits;
         p.keys_per_split = plan.keys_per_split;
-        if (log) log_once(tc ? "prefill_tcgen05" : "prefill_ffma", p, dtype, plan);
-        e = timed(tc ? SDPA_KERNEL_PREFILL_TCGEN05 : SDPA_KERNEL_PREFILL_FFMA, stream, [&] {
-            return tc ? prefill_tc_launch(p, dtype, plan, stream) : ffma_launch(p, dtype, plan, stream);
+        if (log) log_once(tc ? "prefill_tcgen05" : tf ? "prefill_tf32x3" : "prefill_ffma", p, dtype, plan);
+        const int fam = tc ? SDPA_KERNEL_PREFILL_TCGEN05 : tf ? SDPA_KERNEL_PREFILL_TF32 : SDPA_KERNEL_PREFILL_FFMA;
+        e = timed(fam, stream, [&] {
+            return tc ? prefill_tc_launch(p, dtype, plan, stream)
+                      : tf ? prefill_tf32_launch(p, plan, stream) : ffma_launch(p, dtype, plan, stream);
         });
         if (e != cudaSuccess) return cuda_fail(e);
-        (tc ? c_tc : c_pffma).fetch_add(1, std::memory_order_relaxed);
+        (tc ? c_tc : tf ? c_tf32 : c_pffma).fetch_add(1, std::memory_order_relaxed);
         c_prefill.fetch_add(1, std::memory_order_relaxed);
         launches = 1;
     }
@@ -367,6 +429,31 @@ extern "C" int sdpa_forward(const void* q, const void* k, const void* v, void* o
         if (sdpa_check_device_error(stream, &code) != SDPA_OK) return SDPA_ERR_TIMEOUT;
     }
     return SDPA_OK;
+}
+
+}  // namespace
+}  // namespace sdpa
+
+extern "C" int sdpa_forward(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t Hq,
+                            int64_t Hkv, int64_t Lq, int64_t Lk, int64_t Dqk, int64_t Dv,
+                            const int64_t strides[16], float scale, int mask_kind, const void* mask,
+                            const int64_t mask_strides[4], int dtype, void* stream_ptr) {
+    return forward_impl(q, k, v, out, B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, scale, mask_kind, mask, mask_strides,
+                        0, dtype, stream_ptr);
+}
+
+extern "C" int sdpa_forward_window(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t Hq,
+                                   int64_t Hkv, int64_t Lq, int64_t Lk, int64_t Dqk, int64_t Dv,
+                                   const int64_t strides[16], float scale, int64_t window, int dtype,
+                                   void* stream_ptr) {
+    if (window < 1) {
+        c_calls.fetch_add(1, std::memory_order_relaxed);
+        c_rejected.fetch_add(1, std::memory_order_relaxed);
+        t_last_launches = 0;
+        return SDPA_ERR_INVALID_ARG;
+    }
+    return forward_impl(q, k, v, out, B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, scale, SDPA_MASK_SLIDING, nullptr,
+                        nullptr, window, dtype, stream_ptr);
 }
 
 extern "C" const char* sdpa_error_string(int status) {
@@ -400,11 +487,12 @@ extern "C" void sdpa_get_counters(sdpa_counters* out) {
     out->decode_mma_launches = c_dmma.load();
     out->decode_ffma_launches = c_dffma.load();
     out->combine_launches = c_combine.load();
+    out->prefill_tf32_launches = c_tf32.load();
 }
 
 extern "C" void sdpa_reset_counters(void) {
     for (auto* c : {&c_calls, &c_prefill, &c_decode, &c_empty, &c_rejected, &c_tc, &c_pffma, &c_dmma, &c_dffma,
-                    &c_combine})
+                    &c_combine, &c_tf32})
         c->store(0);
 }
 
@@ -415,28 +503,64 @@ extern "C" int sdpa_check_device_error(void* stream_ptr, int* code_out) {
     int code = take_device_error_prefill_tc(stream);
     const int code_d = take_device_error_decode(stream);
     if (code == 0 || code_d < 0) code = code_d;
+    const int code_f = take_device_error_tf32(stream);
+    if (code == 0 || code_f < 0) code = code_f;
     if (code_out) *code_out = code;
     if (code < 0) return SDPA_ERR_CUDA;
-    return code ? SDPA_ERR_TIMEOUT : SDPA_OK;
+    if (code) {
+        // A wait that gave up may have left a split barrier short of its target:
+        // start this stream's next decode call from zeroed counters.
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess) clear_counters(dev, stream);
+        return SDPA_ERR_TIMEOUT;
+    }
+    return SDPA_OK;
+}
+
+extern "C" int sdpa_debug_set(int knob, int64_t value) {
+    switch (knob) {
+        case SDPA_DEBUG_WAIT_LIMIT_NS: g_dbg_wait_limit_ns.store(value); return SDPA_OK;
+        case SDPA_DEBUG_DECODE_BARRIER_EXTRA:
+            if (value < 0 || value > 1024) return SDPA_ERR_INVALID_ARG;
+            g_dbg_barrier_extra.store(value);
+            return SDPA_OK;
+        case SDPA_DEBUG_FAIL_ALLOCS:
+            if (value < 0) return SDPA_ERR_INVALID_ARG;
+            g_dbg_fail_allocs.store(value);
+            return SDPA_OK;
+        default: return SDPA_ERR_INVALID_ARG;
+    }
+}
+
+extern "C" int64_t sdpa_workspace_bytes(void) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    int64_t total = 0;
+    for (auto& kv : g_ws) {
+        total += (int64_t)kv.second.bytes;
+        for (auto& r : kv.second.retired) total += (int64_t)r.second;
+        for (auto& c : kv.second.counters) total += (int64_t)(c.second.second * sizeof(int));
+    }
+    return total;
 }
 
 extern "C" int sdpa_shutdown(void) {
     std::lock_guard<std::mutex> lk(g_mu);
     for (auto& kv : g_ws) {
-        if (kv.second.ptr || kv.second.counters) {
-            int cur = 0;
-            cudaGetDevice(&cur);
-            cudaSetDevice(kv.first.first);
-            cudaFree(kv.second.ptr);   // synchronous: the owning stream may no longer exist
-            if (kv.second.counters) cudaFree(kv.second.counters);
-            cudaSetDevice(cur);
-        }
+        int cur = 0;
+        cudaGetDevice(&cur);
+        cudaSetDevice(kv.first.first);
+        // synchronous frees: the owning stream may no longer exist
+        if (kv.second.ptr) cudaFree(kv.second.ptr);
+        for (auto& r : kv.second.retired) cudaFree(r.first);
+        for (auto& c : kv.second.counters)
+            if (c.second.first) cudaFree(c.second.first);
+        cudaSetDevice(cur);
     }
     g_ws.clear();
     return SDPA_OK;
 }
 
-extern "C" int sdpa_abi_version(void) { return 1; }
+extern "C" int sdpa_abi_version(void) { return 2; }
 
 extern "C" int sdpa_profile_enable(int on) {
     g_prof_on.store(on != 0);

@@ -219,25 +219,29 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t pa
     return ok != 0;
 }
 
-// Bounded wait on an mbarrier phase: about 2 s, then the device error flag is
-// set and false returned.  No wait in this library can spin forever.  The
-// thread sleeps in the barrier between checks of the time limit.
-__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int code) {
+// Bounded wait on an mbarrier phase: `limit_ns` (about 2 s by default), then
+// the device error flag is set and false returned.  No wait in this library
+// can spin forever.  The thread sleeps in the barrier between checks of the
+// time limit.
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int code,
+                                           uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try_wait_suspend(bar, parity, 100000u)) return true;
-        if (globaltimer() - t0 > 2000000000ull) {
+        if (globaltimer() - t0 > limit_ns) {
             atomicCAS(&g_sdpa_device_error, 0, code);
             return false;
         }
     }
 }
 
-// Bounded wait until *counter >= target (a device-scope acquire load), about
-// 2 s, then the device error flag is set and false returned.  Only for
-// counters that CTAs resident at the same time increment.
-__device__ __forceinline__ bool wait_counter_geq(const int* counter, int target, int code) {
+// Bounded wait until *counter >= target (a device-scope acquire load), for
+// `limit_ns` (about 2 s by default), then the device error flag is set and
+// false returned.  Only for counters that CTAs resident at the same time
+// increment.
+__device__ __forceinline__ bool wait_counter_geq(const int* counter, int target, int code,
+                                                 uint64_t limit_ns = kWaitLimitNs) {
     auto load = [&] {
         int v;
         asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
@@ -247,7 +251,7 @@ __device__ __forceinline__ bool wait_counter_geq(const int* counter, int target,
     const uint64_t t0 = globaltimer();
     while (true) {
         if (load() >= target) return true;
-        if (globaltimer() - t0 > 2000000000ull) {
+        if (globaltimer() - t0 > limit_ns) {
             atomicCAS(&g_sdpa_device_error, 0, code);
             return false;
         }

@@ -1,7 +1,6 @@
 // decode_mma.cu -- split-K (flash-decoding) attention for short queries,
 // fp16 / bf16, one launch: TMA loads, warp-level tensor-core MMA (m16n8k16,
-// fp32 accumulation) and a log-sum-exp combine done by the last CTA of each
-// group.
+// fp32 accumulation) and the log-sum-exp merge of the splits.
 //
 // The decode ("vector") path of MLX issue #3885 ("Metal SDPA: no fused path
 // for head_dim=512 ..."), section "Current routing": qL <= 8.  Decode is bound
@@ -12,29 +11,33 @@
 //    heads times the qL queries), so each K/V byte is read once per group
 //    (the MLX commit "Read each K/V byte once in gqa-8 decode attention");
 //  * keys are split across CTAs (split-K) so that B*Hkv small problems still
-//    fill the 148 SMs in one wave; the split count scales with 1/(B*Hkv) (same
-//    issue: its two-pass kernel starves the grid when n_kv is small);
-//  * one producer thread streams 32-key slots of K and V with TMA (128-byte
-//    swizzle, zero fill past Lk; 4 KB boxes, since one thread issuing 2 KB
-//    boxes cannot keep HBM busy) into a CTA-wide ring of NSLOT slots, so about
-//    200 KB are in flight per SM and the consumer warps issue no load
+//    occupy every SM: one CTA per SM, and when the SM count is not a multiple
+//    of the group count the first groups take one split more, so no SM is left
+//    idle (same issue: its two-pass kernel starves the grid when n_kv is small);
+//  * one producer thread streams slots of SK keys of K and V with TMA (128-byte
+//    swizzle, zero fill past Lk; one whole-row box per tensor and slot for head
+//    dims that are multiples of 64) into a CTA-wide ring of ~192 KB, so most of
+//    a CTA's share is requested at once and the consumer warps issue no load
 //    instructions for K and V;
-//  * consumer warp w takes the 16-key sub-blocks w, w+W, ... of the slots;
-//    scores are computed transposed,
-//    S^T = K Q^T, so the keys fill the 16-row side of the MMA and the few query
-//    rows the 8-column side; P^T reaches the B operand of O^T += V^T P^T with
-//    one movmatrix per 8x8 block;
+//  * consumer warp w takes the 16-key sub-blocks w, w+W, ... of the slots; the
+//    additive / boolean mask values of its next sub-block are loaded while it
+//    computes the current one; scores are computed transposed, S^T = K Q^T, so
+//    the keys fill the 16-row side of the MMA and the few query rows the
+//    8-column side; P^T reaches the B operand of O^T += V^T P^T with one
+//    movmatrix per 8x8 block;
 //  * each CTA merges its warps and writes its split's normalised partial and
 //    log-sum-exp; the grid is a cooperative launch (all CTAs resident at once),
 //    so the splits of a (batch, KV head, row group) meet at a bounded barrier
-//    in the workspace and then each merges one slice of the group's output
-//    (one round trip to L2 per CTA instead of one CTA merging everything); the
-//    last CTA to leave resets the barrier, which the library keeps at zero
-//    between calls.
+//    and then each CTA merges its own slice of the group's output, loading
+//    every split's partial of its slice in one round trip.  The barrier is a
+//    64-bit arrival counter per group that only grows: every call adds exactly
+//    S (the group's split count; the workspace keeps separate counters per
+//    launch shape), so a call's target is the next multiple of S above the
+//    value it reads at start.  Arrivals are fire-and-forget reductions and no
+//    CTA needs a second round trip to reset anything.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdlib.h>
-
 
 #include "common.cuh"
 #include "kernels.h"
@@ -77,13 +80,53 @@ struct DecParams {
     AttnParams p;
     MapAxes k_ax, v_ax;
     int RG;          // row groups per KV head
-    int* counters;   // [B * Hkv * RG][2]: arrivals, departures; zero between calls
+    int s_lo;        // splits of a group (the first `extra` groups take one more)
+    int extra;
+    int s_max;       // row stride of the partials (s_lo, or s_lo + 1 when extra > 0)
+    int* counters;   // [B * Hkv * RG] 64-bit arrival counters, multiples of the group's S between calls
 };
 
 // ldmatrix address of 16-byte unit `u` of row `row` in a 128-byte-swizzled chunk.
 __device__ __forceinline__ uint32_t swz(uint32_t chunk, int row, int u) {
     return chunk + (uint32_t)(row * 128 + ((u ^ (row & 7)) << 4));
 }
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// The splits of a group meet here (thread 0 of each CTA; the caller's CTA
+// barrier has ordered every thread's partial stores before it): one
+// fire-and-forget arrival, then a bounded wait for `target` arrivals.  The
+// release (cumulative) publishes this CTA's partials with its arrival; the
+// acquire load that sees the target makes every split's partials visible.
+// Returns false if the wait ran out (device error flag set).
+__device__ __forceinline__ bool split_barrier(unsigned long long* counter, unsigned long long target,
+                                              uint64_t limit_ns) {
+    asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(counter) : "memory");
+    if (ld_acquire_u64(counter) >= target) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        if (ld_acquire_u64(counter) >= target) return true;
+        if (globaltimer() - t0 > limit_ns) {
+            atomicCAS(&g_sdpa_device_error, 0, (int)kErrWaitSplits);
+            return false;
+        }
+    }
+}
+
+template <int NT>
+struct MaskFrag {
+    float add[NT][4];
+    bool keep[NT][4];
+};
 
 template <typename T, int DQK, int DV, int NT, int W, int NSLOT, int SK>
 __global__ void __launch_bounds__((W + 1) * 32, 1)
@@ -106,9 +149,26 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g8 = lane >> 2, t4 = lane & 3;   // MMA fragment coordinates
-    const int split = blockIdx.x;
-    const int hkv = blockIdx.y / dp.RG, rg = blockIdx.y % dp.RG;
-    const int b = blockIdx.z;
+
+    // ---- which group and split this CTA serves
+    int grp, split, S;
+    {
+        const int c = (int)blockIdx.x;
+        const int big = dp.extra * (dp.s_lo + 1);
+        if (c < big) {
+            grp = c / (dp.s_lo + 1);
+            split = c - grp * (dp.s_lo + 1);
+            S = dp.s_lo + 1;
+        } else {
+            const int c2 = c - big;
+            grp = dp.extra + c2 / dp.s_lo;
+            split = c2 - (c2 / dp.s_lo) * dp.s_lo;
+            S = dp.s_lo;
+        }
+    }
+    const int rg = grp % dp.RG;
+    const int hkv = (grp / dp.RG) % (int)p.Hkv;
+    const int b = grp / (dp.RG * (int)p.Hkv);
     const int64_t G = p.group, R = G * p.Lq;
     const int64_t row0 = (int64_t)rg * C::ROWS;
 
@@ -124,51 +184,43 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         tma_prefetch_desc(&tmK);   // kernel parameters: safe before the wait below
         tma_prefetch_desc(&tmV);
     }
+
+    // ---- slots of this split (SK keys each): the keys any row of the CTA can
+    // see (all of them; up to the causal horizon; inside the sliding window)
+    // are divided among the group's S splits
+    int64_t key_first = 0, key_last = p.Lk - 1;
+    if (p.mask_kind == 3 || p.mask_kind == 4) {
+        int64_t max_i = -1, min_i = p.Lq;   // query indices among this CTA's rows
+        for (int r = 0; r < C::ROWS; ++r)
+            if (row0 + r < R) {
+                max_i = max(max_i, (row0 + r) % p.Lq);
+                min_i = min(min_i, (row0 + r) % p.Lq);
+            }
+        key_last = min(key_last, max_i + p.Lk - p.Lq);   // last key any row sees
+        if (p.mask_kind == 4) key_first = max(key_first, min_i + p.Lk - p.Lq - p.window + 1);
+    }
+    int64_t sl_begin = 0, sl_end = 0;
+    if (key_last >= key_first) {
+        const int64_t sl_first = key_first / SK, nv = key_last / SK + 1 - sl_first;
+        sl_begin = sl_first + nv * split / S;
+        sl_end = sl_first + nv * (split + 1) / S;
+    }
+    const int n_slots = sl_end > sl_begin ? (int)(sl_end - sl_begin) : 0;
+
     // Inputs and the split counters may come from the previous kernel of the
     // stream: wait for it to complete before the first global access.
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    // the group's arrival counter, read now (its round trip is then off the
+    // path after the partials): every call on it adds exactly S, and no CTA of
+    // this call can have arrived S times yet, so this call's target is the next
+    // multiple of S
+    unsigned long long* ctr = reinterpret_cast<unsigned long long*>(dp.counters) + grp;
+    unsigned long long target = 0;
+    if (tid == 0 && S > 1) {
+        const unsigned long long c0 = ld_relaxed_u64(ctr);
+        target = c0 - c0 % (unsigned long long)S + (unsigned long long)S + (unsigned long long)p.barrier_extra;
+    }
     __syncthreads();   // barriers initialised; the producer starts streaming K/V right away
-    if (warp > 0) {
-        // ---- Q rows of this CTA (zero rows past the group and zero pad columns), consumer warps only
-        const T* qg = reinterpret_cast<const T*>(p.q);
-        constexpr int CH = C::DQKP / 8;   // 16-byte chunks per padded row
-        for (int idx = tid - 32; idx < C::ROWS * CH; idx += C::THREADS - 32) {
-            const int r = idx / CH, c = idx % CH;
-            const int64_t gr = row0 + r;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (gr < R && c * 8 < DQK) {
-                const int64_t h = hkv * G + gr / p.Lq, i = gr % p.Lq;
-                val = *reinterpret_cast<const uint4*>(qg + b * p.sq[0] + h * p.sq[1] + i * p.sq[2] + c * 8);
-            }
-            *reinterpret_cast<uint4*>(Qs + r * C::QS + c * 8) = val;
-        }
-        for (int r = tid - 32; r < C::ROWS; r += C::THREADS - 32) {   // per-row output / partial offsets
-            const int64_t gr = row0 + r;
-            if (gr < R) {
-                const int64_t h = hkv * G + gr / p.Lq, i = gr % p.Lq;
-                row_out[r] = b * p.so[0] + h * p.so[1] + i * p.so[2];
-                row_part[r] = ((int64_t)b * p.Hq + h) * p.Lq + i;
-            } else {
-                row_out[r] = 0;
-                row_part[r] = -1;
-            }
-        }
-        asm volatile("bar.sync 1, %0;\n" ::"n"(W * 32) : "memory");   // consumer warps only
-    }
-
-    // ---- slots of this split (SK keys each), cut at the causal horizon
-    const int64_t nsl = (p.Lk + SK - 1) / SK;
-    const int64_t slps = p.keys_per_split / SK;
-    const int64_t sl_begin = (int64_t)split * slps;
-    int64_t sl_end = min(nsl, sl_begin + slps);
-    if (p.mask_kind == 3) {
-        int64_t max_i = -1;   // largest query index among this CTA's rows
-        for (int r = 0; r < C::ROWS; ++r)
-            if (row0 + r < R) max_i = max(max_i, (row0 + r) % p.Lq);
-        const int64_t last = max_i + p.Lk - p.Lq;   // last key any row sees
-        sl_end = min(sl_end, last < 0 ? (int64_t)0 : last / SK + 1);
-    }
-    const int n_slots = sl_end > sl_begin ? (int)(sl_end - sl_begin) : 0;
 
     // per-thread state: rows (nt*8 + 2*t4 + {0,1}); O^T fragments (consumer warps)
     float m_run[NT][2], l_run[NT][2];
@@ -192,7 +244,9 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
             bool ok = true;
             for (; t < n_slots; ++t) {
                 const int slot = t % NSLOT;
-                if (!(ok = wait_phase(bar_empty + slot, ((t / NSLOT) & 1) ^ 1, kErrWaitSlot))) break;
+                if (t >= NSLOT &&
+                    !(ok = wait_phase(bar_empty + slot, ((t / NSLOT) & 1) ^ 1, kErrWaitSlot, p.wait_limit_ns)))
+                    break;
                 mbar_arrive_expect_tx(bar_full + slot, C::SLOT);
                 const int key0 = (int)((sl_begin + t) * SK);
                 const uint32_t base = ring + slot * C::SLOT;
@@ -214,10 +268,35 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
             }
             if (!ok)   // every issued load must land before shared memory is reused or released
                 for (int x = (t > NSLOT ? t - NSLOT : 0); x < t; ++x)
-                    wait_phase(bar_full + x % NSLOT, (x / NSLOT) & 1, kErrWaitTmaLoad);
+                    wait_phase(bar_full + x % NSLOT, (x / NSLOT) & 1, kErrWaitTmaLoad, p.wait_limit_ns);
         }
     } else {
         // ------------------------------------------------------------ consumer warps
+        // Q rows of this CTA (zero rows past the group and zero pad columns)
+        const T* qg = reinterpret_cast<const T*>(p.q);
+        constexpr int CH = C::DQKP / 8;   // 16-byte chunks per padded row
+        for (int idx = tid - 32; idx < C::ROWS * CH; idx += C::THREADS - 32) {
+            const int r = idx / CH, c = idx % CH;
+            const int64_t gr = row0 + r;
+            uint4 val = make_uint4(0, 0, 0, 0);
+            if (gr < R && c * 8 < DQK) {
+                const int64_t h = hkv * G + gr / p.Lq, i = gr % p.Lq;
+                val = *reinterpret_cast<const uint4*>(qg + b * p.sq[0] + h * p.sq[1] + i * p.sq[2] + c * 8);
+            }
+            *reinterpret_cast<uint4*>(Qs + r * C::QS + c * 8) = val;
+        }
+        for (int r = tid - 32; r < C::ROWS; r += C::THREADS - 32) {   // per-row output / partial offsets
+            const int64_t gr = row0 + r;
+            if (gr < R) {
+                const int64_t h = hkv * G + gr / p.Lq, i = gr % p.Lq;
+                row_out[r] = b * p.so[0] + h * p.so[1] + i * p.so[2];
+                row_part[r] = ((int64_t)b * p.Hq + h) * p.Lq + i;
+            } else {
+                row_out[r] = 0;
+                row_part[r] = -1;
+            }
+        }
+
         const int w = warp - 1;
         int64_t row_h[NT][2], row_i[NT][2];
         bool row_ok[NT][2];
@@ -230,17 +309,10 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                 row_h[nt][c] = hkv * G + (gr < R ? gr / p.Lq : 0);
                 row_i[nt][c] = gr < R ? gr % p.Lq : 0;
             }
-        const uint32_t q_base = smem_u32(Qs);
         const float log2e = 1.4426950408889634f;
-        const int mi = lane >> 3;   // which 8x8 matrix this lane addresses in an x4 ldmatrix
-
-        for (int item = w; item < n_slots * kNSUB; item += W) {
-            const int t = item / kNSUB, u = item % kNSUB;   // slot t, 16-key sub-block u
-            const int slot = t % NSLOT;
-            const int64_t kb = (sl_begin + t) * kNSUB + u;   // global 16-key block index
-            // mask values of this block, loaded before waiting for K/V so the two latencies overlap
-            float madd[NT][4];
-            bool mkeep[NT][4];
+        // mask values of one 16-key sub-block; s[nt][c] holds key g8 + 8*(c>>1), row 2*t4 + (c&1)
+        auto load_mask = [&](int item, MaskFrag<NT>& mf) {
+            const int64_t kb = (sl_begin + item / kNSUB) * kNSUB + item % kNSUB;   // global 16-key block
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -249,7 +321,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                     const int64_t j = kb * 16 + g8 + 8 * (c >> 1);
                     bool keep = row_ok[nt][rc] && j < p.Lk;
                     float add = 0.f;
-                    if (keep && p.mask_kind != 0 && p.mask_kind != 3) {
+                    if (keep && (p.mask_kind == 1 || p.mask_kind == 2)) {   // a mask tensor to read
                         const int64_t moff =
                             b * p.sm[0] + row_h[nt][rc] * p.sm[1] + row_i[nt][rc] * p.sm[2] + j * p.sm[3];
                         if (p.mask_kind == 1)
@@ -258,11 +330,39 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                             keep = reinterpret_cast<const uint8_t*>(p.mask)[moff] != 0;
                     } else if (keep && p.mask_kind == 3) {
                         keep = j <= row_i[nt][rc] + p.Lk - p.Lq;
+                    } else if (keep && p.mask_kind == 4) {
+                        const int64_t own = row_i[nt][rc] + p.Lk - p.Lq;
+                        keep = j <= own && j > own - p.window;
                     }
-                    madd[nt][c] = add;
-                    mkeep[nt][c] = keep;
+                    mf.add[nt][c] = add;
+                    mf.keep[nt][c] = keep;
                 }
-            if (!__all_sync(0xffffffffu, wait_phase(bar_full + slot, (t / NSLOT) & 1, kErrWaitTmaLoad))) break;
+        };
+        const int n_items = n_slots * kNSUB;
+        // one sub-block ahead where the registers allow (NT <= 2); with 32 rows
+        // per CTA the values load right before the wait for the sub-block's data
+        constexpr bool kAhead = NT <= 2;
+        MaskFrag<NT> mnext;
+        if (kAhead && w < n_items) load_mask(w, mnext);
+        asm volatile("bar.sync 1, %0;\n" ::"n"(W * 32) : "memory");   // Q and row offsets written (consumers)
+
+        const uint32_t q_base = smem_u32(Qs);
+        const int mi = lane >> 3;   // which 8x8 matrix this lane addresses in an x4 ldmatrix
+
+        for (int item = w; item < n_items; item += W) {
+            const int t = item / kNSUB, u = item % kNSUB;   // slot t, 16-key sub-block u
+            const int slot = t % NSLOT;
+            MaskFrag<NT> mcur;
+            if (kAhead) {
+                mcur = mnext;
+                // the next sub-block's mask values load while this one computes
+                if (item + W < n_items) load_mask(item + W, mnext);
+            } else {
+                load_mask(item, mcur);
+            }
+            if (!__all_sync(0xffffffffu, wait_phase(bar_full + slot, (t / NSLOT) & 1, kErrWaitTmaLoad,
+                                                    p.wait_limit_ns)))
+                break;
             const uint32_t kbase = ring + slot * C::SLOT;
             const uint32_t vbase = kbase + C::NBK * kChunk;
             const int rsub = u * 16;   // first row of this sub-block inside the slot
@@ -296,14 +396,14 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                     for (int c = 0; c < 4; ++c) s[nt][c] += s2[nt][c];
             }
 
-            // scale, mask, online softmax (log2 domain).  s[nt][c]: key g8 + 8*(c>>1), row 2*t4 + (c&1)
+            // scale, mask, online softmax (log2 domain)
             uint32_t pb[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 float bmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const float x = mkeep[nt][c] ? fmaf(s[nt][c], p.scale_log2, madd[nt][c]) : -INFINITY;
+                    const float x = mcur.keep[nt][c] ? fmaf(s[nt][c], p.scale_log2, mcur.add[nt][c]) : -INFINITY;
                     s[nt][c] = x;
                     bmax[c & 1] = fmaxf(bmax[c & 1], x);
                 }
@@ -389,9 +489,9 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     }
     __syncthreads();
 
-    const int S = p.splits;
+    const int n_rows = (int)min((int64_t)C::ROWS, R - row0);   // real query rows of this CTA
     float* coef = reinterpret_cast<float*>(smem + C::OFF_COEF);   // [ROWS][W + 1]
-    for (int r = tid; r < C::ROWS; r += C::THREADS) {           // per row: weights of the W warps, lse
+    for (int r = tid; r < n_rows; r += C::THREADS) {            // per row: weights of the W warps, lse
         float mmax = -INFINITY;
 #pragma unroll
         for (int w = 0; w < W; ++w) mmax = fmaxf(mmax, merge[((size_t)w * C::ROWS + r) * C::MS + C::DVP]);
@@ -408,10 +508,10 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         coef[r * (W + 1) + W] = (L > 0.f) ? mmax + log2f(L) : -INFINITY;
     }
     __syncthreads();
-    for (int idx = tid; idx < C::ROWS * (DV / 4); idx += C::THREADS) {
+    const int SM = dp.s_max;
+    for (int idx = tid; idx < n_rows * (DV / 4); idx += C::THREADS) {
         const int r = idx / (DV / 4), c4 = idx % (DV / 4);
         const int64_t row = row_part[r];
-        if (row < 0) continue;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int w = 0; w < W; ++w) {
@@ -428,81 +528,69 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
             pk.y = pack2<T>(acc.z, acc.w);
             *reinterpret_cast<uint2*>(reinterpret_cast<T*>(p.out) + row_out[r] + c4 * 4) = pk;
         } else {
-            __stcg(reinterpret_cast<float4*>(p.part_o + (row * S + split) * DV) + c4, acc);
-            if (c4 == 0) __stcg(p.part_lse + row * S + split, coef[r * (W + 1) + W]);
+            __stcg(reinterpret_cast<float4*>(p.part_o + (row * SM + split) * DV) + c4, acc);
+            if (c4 == 0) __stcg(p.part_lse + row * SM + split, coef[r * (W + 1) + W]);
         }
     }
     if (S == 1) return;
 
-    // ---- the S splits of this (batch, KV head, row group) meet: arrivals are
-    // counted in the workspace (every CTA of the grid is resident: cooperative
-    // launch), then each CTA merges its slice of the group's rows x columns
-    int* counter = dp.counters + (((int64_t)b * p.Hkv + hkv) * dp.RG + rg) * 2;
-    // The CTA barrier orders every thread's partial stores before thread 0's
-    // arrival, whose release (cumulative) makes them visible with it.
+    // ---- the S splits of this group meet (every CTA of the grid is resident:
+    // cooperative launch), then each CTA merges its slice of the group's rows x
+    // columns.  The CTA barrier orders every thread's partial stores before
+    // thread 0's arrival, whose release (cumulative) makes them visible with it.
     __syncthreads();
-    if (tid == 0) {
-        asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(counter) : "memory");
-        *s_flag = wait_counter_geq(counter, S, kErrWaitSplits) ? 1 : 0;
-    }
+    if (tid == 0)
+        *s_flag = split_barrier(ctr, target, p.wait_limit_ns) ? 1 : 0;
     __syncthreads();
-    if (*s_flag) {
-        // this split's share of the (row, 4-column) items; each thread merges
-        // its items online over the splits, 16 splits (their log-sum-exps and
-        // partials) in flight per round trip
-        const int items = C::ROWS * (DV / 4);
-        const int per = (items + S - 1) / S;
-        const int i_end = min(items, (split + 1) * per);
-        for (int idx = split * per + tid; idx < i_end; idx += C::THREADS) {
-            const int r = idx / (DV / 4), c4 = idx % (DV / 4);
-            const int64_t row = row_part[r];
-            if (row < 0) continue;
-            const float4* po = reinterpret_cast<const float4*>(p.part_o + row * S * DV) + c4;
-            const float* pl = p.part_lse + row * S;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            float mx = -INFINITY, sum = 0.f;
-            for (int s0 = 0; s0 < S; s0 += 16) {
-                float lse[16];
-                float4 v[16];
+    if (!*s_flag) return;
+    // this split's share of the (row, 4-column) items; each thread merges its
+    // items online over the splits, 32 splits (their log-sum-exps and
+    // partials) in flight per round trip
+    const int items = n_rows * (DV / 4);
+    const int per = (items + S - 1) / S;
+    const int i_end = min(items, (split + 1) * per);
+    for (int idx = split * per + tid; idx < i_end; idx += C::THREADS) {
+        const int r = idx / (DV / 4), c4 = idx % (DV / 4);
+        const int64_t row = row_part[r];
+        const float4* po = reinterpret_cast<const float4*>(p.part_o + row * SM * DV) + c4;
+        const float* pl = p.part_lse + row * SM;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float mx = -INFINITY, sum = 0.f;
+        for (int s0 = 0; s0 < S; s0 += 32) {
+            float lse[32];
+            float4 v[32];
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const bool in = s0 + u < S;
-                    lse[u] = in ? __ldcg(pl + s0 + u) : -INFINITY;
-                    v[u] = in ? __ldcg(po + (int64_t)(s0 + u) * (DV / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-                float cm = mx;
-#pragma unroll
-                for (int u = 0; u < 16; ++u) cm = fmaxf(cm, lse[u]);
-                if (cm == -INFINITY) continue;   // no key of these splits is visible
-                const float f = (mx == -INFINITY) ? 0.f : fast_exp2(mx - cm);
-                acc.x *= f;
-                acc.y *= f;
-                acc.z *= f;
-                acc.w *= f;
-                sum *= f;
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const float ws = (lse[u] == -INFINITY) ? 0.f : fast_exp2(lse[u] - cm);
-                    sum += ws;
-                    acc.x = fmaf(ws, v[u].x, acc.x);
-                    acc.y = fmaf(ws, v[u].y, acc.y);
-                    acc.z = fmaf(ws, v[u].z, acc.z);
-                    acc.w = fmaf(ws, v[u].w, acc.w);
-                }
-                mx = cm;
+            for (int u = 0; u < 32; ++u) {
+                const bool in = s0 + u < S;
+                lse[u] = in ? __ldcg(pl + s0 + u) : -INFINITY;
+                v[u] = in ? __ldcg(po + (int64_t)(s0 + u) * (DV / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
-            uint2 pk;
-            pk.x = pack2<T>(acc.x * inv, acc.y * inv);
-            pk.y = pack2<T>(acc.z * inv, acc.w * inv);
-            *reinterpret_cast<uint2*>(reinterpret_cast<T*>(p.out) + row_out[r] + c4 * 4) = pk;
+            float cm = mx;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) cm = fmaxf(cm, lse[u]);
+            if (cm == -INFINITY) continue;   // no key of these splits is visible
+            const float f = (mx == -INFINITY) ? 0.f : fast_exp2(mx - cm);
+            acc.x *= f;
+            acc.y *= f;
+            acc.z *= f;
+            acc.w *= f;
+            sum *= f;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                const float ws = (lse[u] == -INFINITY) ? 0.f : fast_exp2(lse[u] - cm);
+                sum += ws;
+                acc.x = fmaf(ws, v[u].x, acc.x);
+                acc.y = fmaf(ws, v[u].y, acc.y);
+                acc.z = fmaf(ws, v[u].z, acc.z);
+                acc.w = fmaf(ws, v[u].w, acc.w);
+            }
+            mx = cm;
         }
-    }
-    // the last split to leave resets the barrier for the next call on this workspace
-    __syncthreads();
-    if (tid == 0 && atomicAdd(counter + 1, 1) == S - 1) {
-        counter[0] = 0;
-        counter[1] = 0;
+        const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
+        uint2 pk;
+        pk.x = pack2<T>(acc.x * inv, acc.y * inv);
+        pk.y = pack2<T>(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2*>(reinterpret_cast<T*>(p.out) + row_out[r] + c4 * 4) = pk;
     }
 }
 
@@ -522,14 +610,14 @@ Shape shape_of() {
 // NT in {1, 2, 4} with the O^T accumulators at DVP*NT/4 registers per
 // thread (NT = 1 only at Dv = 512, NT <= 2 at Dv = 256).
 #define SDPA_DECODE_DIMS(X) \
-    X(64, 64, 4, 12, 64)    \
-    X(72, 72, 4, 6, 64)     \
-    X(80, 80, 4, 6, 64)     \
-    X(96, 96, 4, 6, 64)     \
-    X(128, 128, 4, 6, 64)   \
-    X(192, 128, 4, 5, 64)   \
-    X(256, 256, 4, 6, 32)   \
-    X(512, 512, 4, 3, 32)
+    X(64, 64, 7, 12, 64)    \
+    X(72, 72, 7, 6, 64)     \
+    X(80, 80, 7, 6, 64)     \
+    X(96, 96, 7, 6, 64)     \
+    X(128, 128, 7, 6, 64)   \
+    X(192, 128, 7, 5, 64)   \
+    X(256, 256, 7, 6, 32)   \
+    X(512, 512, 7, 3, 32)
 
 constexpr int nt_cap(int dv) { return dv >= 512 ? 1 : (dv >= 256 ? 2 : 4); }
 constexpr int nt_fix(int want, int dv) { return want < nt_cap(dv) ? want : nt_cap(dv); }
@@ -604,44 +692,66 @@ bool decode_mma_supported(int dtype, int64_t Dqk, int64_t Dv) {
     return (dtype == 1 || dtype == 2) && pick_shape(Dqk, Dv, 8).smem != 0;
 }
 
-// Work split.  A (batch, KV head, row group) is a group; its keys are split
-// across `splits` CTAs so that the grid fills the SMs in one wave (one CTA per
-// SM: the kernel takes most of the shared memory).
+// Work split.  A (batch, KV head, row group) is a group; its slots of keys are
+// split across CTAs so that the grid has one CTA per SM (the kernel takes most
+// of the shared memory): with `groups` groups on `sm` SMs, the first sm % groups
+// groups take sm / groups + 1 splits and the others sm / groups, each split at
+// most one slot short of the others.  More groups than SMs: one CTA per group,
+// in waves.  A head-dim pair this kernel does not cover gets an empty grid,
+// which every caller refuses.
 LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev) {
     (void)dtype;
     LaunchPlan plan{};
     const int64_t rows = (int64_t)p.group * p.Lq;
     const Shape sh = pick_shape(p.Dqk, p.Dv, rows);
+    if (sh.smem == 0 || rows <= 0 || p.B <= 0 || p.Hkv <= 0) return plan;
     const int64_t RG = (rows + 8 * sh.nt - 1) / (8 * sh.nt);
-    const int64_t nkb = (p.Lk + sh.sk - 1) / sh.sk;   // slots of sh.sk keys
-    const int64_t base = p.B * p.Hkv * RG;
-    const int nsub = sh.sk / 16;
-    const int64_t max_splits = (nkb * nsub + sh.w - 1) / sh.w;   // at least one sub-block per consumer warp
-    int64_t splits = (int64_t)dev.sm_count / base;   // one CTA per SM, one wave
-    if (splits > max_splits) splits = max_splits;
-    if (splits > kMaxSplits - 1) splits = kMaxSplits - 1;
-    if (splits < 1) splits = 1;
-    // debugging override; a grid that cannot be resident at once makes the
-    // cooperative launch fail with an error
+    // slots of sh.sk keys per group that some row may see (a sliding window
+    // covers at most window + Lq - 1 keys, which may straddle one more slot)
+    int64_t nsl = (p.Lk + sh.sk - 1) / sh.sk;
+    if (p.mask_kind == 4) {
+        const int64_t vis = p.window + p.Lq - 1 < p.Lk ? p.window + p.Lq - 1 : p.Lk;
+        const int64_t nsl_vis = (vis + sh.sk - 1) / sh.sk + 1;
+        if (nsl_vis < nsl) nsl = nsl_vis;
+    }
+    const int64_t groups = p.B * p.Hkv * RG;
+    int64_t lo = 1, extra = 0;
+    if (groups < dev.sm_count) {
+        lo = dev.sm_count / groups;
+        extra = dev.sm_count % groups;
+        if (lo >= nsl) {   // every split gets at least one slot
+            lo = nsl > 0 ? nsl : 1;
+            extra = 0;
+        }
+        if (lo + (extra > 0) > kMaxSplits - 1) {
+            lo = kMaxSplits - 1;
+            extra = 0;
+        }
+    }
+    // debugging override: the same number of splits for every group; a grid
+    // that cannot be resident at once makes the cooperative launch fail
     if (const char* env = getenv("SDPA_DECODE_SPLITS")) {
         const long v = strtol(env, nullptr, 10);
-        if (v >= 1) splits = v < kMaxSplits - 1 ? v : kMaxSplits - 1;
+        if (v >= 1) {
+            lo = v < kMaxSplits - 1 ? v : kMaxSplits - 1;
+            extra = 0;
+        }
     }
-    int64_t kbps = (nkb + splits - 1) / splits;
-    if (kbps < 1) kbps = 1;
-    splits = (nkb + kbps - 1) / kbps;
-    if (splits < 1) splits = 1;
-    plan.grid = dim3((unsigned)splits, (unsigned)(p.Hkv * RG), (unsigned)p.B);
+    const int64_t ctas = groups * lo + extra;
+    if (ctas > 0x7fffffff) return plan;
+    plan.grid = dim3((unsigned)ctas, 1, 1);
     plan.block = dim3((unsigned)((sh.w + 1) * 32), 1, 1);
     plan.smem_bytes = sh.smem;
-    plan.splits = (int)splits;
-    plan.keys_per_split = kbps * sh.sk;
+    plan.splits = (int)(lo + (extra > 0));
+    plan.split_lo = (int)lo;
+    plan.split_extra = (int)extra;
+    plan.keys_per_split = ((nsl + lo - 1) / lo) * sh.sk;   // the largest split (informational)
     plan.variant = (int)RG;
     plan.aux = sh.nt;
     return plan;
 }
 
-
+// ints of counter space (one 64-bit counter per group)
 size_t decode_mma_counters(const AttnParams& p, const LaunchPlan& plan) {
     return (size_t)p.B * p.Hkv * plan.variant * 2;
 }
@@ -649,9 +759,14 @@ size_t decode_mma_counters(const AttnParams& p, const LaunchPlan& plan) {
 cudaError_t decode_mma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, int* counters,
                               cudaStream_t stream) {
     if (plan.splits > 1 && (plan.splits >= kMaxSplits || counters == nullptr)) return cudaErrorInvalidValue;
+    if (plan.split_lo < 1 || plan.splits != plan.split_lo + (plan.split_extra > 0 ? 1 : 0))
+        return cudaErrorInvalidValue;
     DecParams dp{};
     dp.p = p;
     dp.RG = plan.variant;
+    dp.s_lo = plan.split_lo;
+    dp.extra = plan.split_extra;
+    dp.s_max = plan.splits;
     dp.counters = counters;
     const int sk = pick_shape(p.Dqk, p.Dv, (int64_t)p.group * p.Lq).sk;
     CUtensorMap mk, mv;

@@ -113,17 +113,24 @@ __global__ void __launch_bounds__(kThreads) flash_ffma_kernel(const AttnParams p
     }
 
     // Key range of this CTA: its split, cut at the last key any of its rows can see.
-    int64_t k_begin = (int64_t)split * p.keys_per_split;
+    int64_t k_begin = p.key_begin + (int64_t)split * p.keys_per_split;
     int64_t k_end = k_begin + p.keys_per_split;
     if (k_end > p.Lk) k_end = p.Lk;
-    if (p.mask_kind == 3) {  // causal, bottom-right: key j visible to query i iff j <= i + Lk - Lq
-        int64_t max_i = -1;
+    if (p.mask_kind == 3 || p.mask_kind == 4) {  // causal, bottom-right: key j visible to query i iff j <= i + Lk - Lq
+        int64_t max_i = -1, min_i = p.Lq;
         for (int rr = 0; rr < kRT; ++rr) {
             const int64_t g2 = row0 + rr;
-            if (g2 < R) max_i = max(max_i, g2 % p.Lq);
+            if (g2 < R) {
+                max_i = max(max_i, g2 % p.Lq);
+                min_i = min(min_i, g2 % p.Lq);
+            }
         }
         const int64_t last = max_i + p.Lk - p.Lq;
         if (k_end > last + 1) k_end = last + 1;
+        if (p.mask_kind == 4) {   // sliding window: nothing before the first row's window
+            const int64_t first = min_i + p.Lk - p.Lq - p.window + 1;
+            if (k_begin < first) k_begin = first;
+        }
     }
 
     float m = -INFINITY;   // running max (log2 domain), identical in the row's 8 threads
@@ -163,6 +170,8 @@ __global__ void __launch_bounds__(kThreads) flash_ffma_kernel(const AttnParams p
                 keep = mp[b * p.sm[0] + hq * p.sm[1] + qi * p.sm[2] + j * p.sm[3]] != 0;
             } else if (keep && p.mask_kind == 3) {
                 keep = j <= qi + p.Lk - p.Lq;
+            } else if (keep && p.mask_kind == 4) {
+                keep = j <= qi + p.Lk - p.Lq && j > qi + p.Lk - p.Lq - p.window;
             }
             if (!keep) s[u] = -INFINITY;
             tmax = fmaxf(tmax, s[u]);
@@ -330,16 +339,24 @@ __global__ void __launch_bounds__(kTThreads, MINB) flash_tiled_f32_kernel(const 
     const float* kg = reinterpret_cast<const float*>(p.k) + b * p.sk[0] + hkv * p.sk[1];
     const float* vg = reinterpret_cast<const float*>(p.v) + b * p.sv[0] + hkv * p.sv[1];
 
-    // Key range: all keys, cut for causal at the last key any row of the CTA sees.
-    int64_t k_end = p.Lk;
-    if (MASK == 3) {
+    // Key range: all keys, cut for causal (and sliding-window) masks at the
+    // last key any row of the CTA sees, and for a sliding window started at
+    // the first key any row sees.
+    int64_t k_begin = 0, k_end = p.Lk;
+    if (MASK == 3 || MASK == 4) {
         const int64_t last_row = min(row0 + kTM, R) - 1;
         // rows of the CTA may span two heads; the largest query index is Lq-1
-        // unless all rows sit in one head
-        const int64_t max_i = (row0 / p.Lq == last_row / p.Lq) ? last_row % p.Lq : p.Lq - 1;
+        // (the smallest 0) unless all rows sit in one head
+        const bool one_head = row0 / p.Lq == last_row / p.Lq;
+        const int64_t max_i = one_head ? last_row % p.Lq : p.Lq - 1;
         k_end = min(k_end, max_i + p.Lk - p.Lq + 1);
+        if (MASK == 4) {
+            const int64_t min_i = one_head ? row0 % p.Lq : 0;
+            k_begin = max((int64_t)0, min_i + p.Lk - p.Lq - p.window + 1);
+        }
     }
-    if (k_end > 0) tiled_issue_rows<DQK, S::KS>(Ks, kg, p.sk[2], (int)min((int64_t)kTN, k_end));
+    if (k_end > k_begin)
+        tiled_issue_rows<DQK, S::KS>(Ks, kg + k_begin * p.sk[2], p.sk[2], (int)min((int64_t)kTN, k_end - k_begin));
 
     // Qt: 32 consecutive rows per warp and one 4-column chunk, so each
     // transposed store is 32 consecutive floats.
@@ -379,7 +396,7 @@ __global__ void __launch_bounds__(kTThreads, MINB) flash_tiled_f32_kernel(const 
     }
     const float log2e = 1.4426950408889634f;
 
-    for (int64_t kt = 0; kt < k_end; kt += kTN) {
+    for (int64_t kt = k_begin; kt < k_end; kt += kTN) {
         const int nvalid = (int)min((int64_t)kTN, k_end - kt);
         cp_async_wait<0>();   // K of this tile (the only group in flight)
         __syncthreads();      // K (and Qt) visible; the previous P.V is done with V and Pt
@@ -425,7 +442,8 @@ __global__ void __launch_bounds__(kTThreads, MINB) flash_tiled_f32_kernel(const 
                         s[i][k] += __ldg(reinterpret_cast<const float*>(p.mask) + moff[i] + j * p.sm[3]) * log2e;
                     if (MASK == 2 && keep)
                         keep = __ldg(reinterpret_cast<const uint8_t*>(p.mask) + moff[i] + j * p.sm[3]) != 0;
-                    if (MASK == 3) keep = keep && j <= qi[i] + p.Lk - p.Lq;
+                    if (MASK == 3 || MASK == 4) keep = keep && j <= qi[i] + p.Lk - p.Lq;
+                    if (MASK == 4) keep = keep && j > qi[i] + p.Lk - p.Lq - p.window;
                     if (!keep) s[i][k] = -INFINITY;
                 }
         }
@@ -521,6 +539,7 @@ cudaError_t launch_tiled(const AttnParams& p, const LaunchPlan& plan, cudaStream
         case 1: return launch_tiled_mask<DQK, DV, 1>(p, plan, s);
         case 2: return launch_tiled_mask<DQK, DV, 2>(p, plan, s);
         case 3: return launch_tiled_mask<DQK, DV, 3>(p, plan, s);
+        case 4: return launch_tiled_mask<DQK, DV, 4>(p, plan, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -619,7 +638,7 @@ LaunchPlan ffma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev, bool
         // Fill the SMs: split the keys until there are about two CTAs per SM,
         // keeping at least two key tiles per split.
         const int64_t base = row_tiles * p.Hkv * p.B;
-        const int64_t tiles = (p.Lk + kKT - 1) / kKT;
+        const int64_t tiles = (p.Lk - p.key_begin + kKT - 1) / kKT;
         int64_t want = (2 * (int64_t)dev.sm_count + base - 1) / base;
         int64_t cap = (tiles + 1) / 2;
         if (want > cap) want = cap;
@@ -627,10 +646,11 @@ LaunchPlan ffma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev, bool
         if (want < 1) want = 1;
         splits = (int)want;
     }
-    int64_t kps = (p.Lk + splits - 1) / splits;
+    const int64_t span = p.Lk - p.key_begin;        // keys any query may see
+    int64_t kps = (span + splits - 1) / splits;
     kps = ((kps + kKT - 1) / kKT) * kKT;            // whole key tiles per split
     if (kps < kKT) kps = kKT;
-    splits = (int)((p.Lk + kps - 1) / kps);
+    splits = (int)((span + kps - 1) / kps);
     if (splits < 1) splits = 1;
     plan.grid = dim3((unsigned)row_tiles, (unsigned)p.Hkv, (unsigned)(p.B * splits));
     plan.block = dim3(kThreads);

@@ -59,15 +59,13 @@ int noalloc_device(int dev, NoallocDevice* out) {
     auto it = g_na_devices.find(dev);
     if (it == g_na_devices.end()) {
         NoallocDevice d;
-        if (cudaGetSymbolAddress(&d.scratch, g_noalloc_scratch) != cudaSuccess || d.scratch == nullptr) {
-            cudaGetLastError();
-            return SDPA_ERR_CUDA;
-        }
-        if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
-            cudaGetLastError();
-            return SDPA_ERR_CUDA;
-        }
+        cudaError_t e = cudaGetSymbolAddress(&d.scratch, g_noalloc_scratch);
+        if (e != cudaSuccess) return record_cuda_error(e);
+        if (d.scratch == nullptr) return record_cuda_error(cudaErrorInvalidSymbol);
+        if ((e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+                cudaSuccess)
+            return record_cuda_error(e);
         it = g_na_devices.emplace(dev, d).first;
     }
     *out = it->second;
@@ -90,16 +88,21 @@ extern "C" int sdpa_forward_noalloc(const void* q, const void* k, const void* v,
     if (!(scale == scale) || scale > 3.4e38f || scale < -3.4e38f) return SDPA_ERR_INVALID_ARG;
     const bool needs_mask = (mask_kind == SDPA_MASK_ADDITIVE || mask_kind == SDPA_MASK_BOOL);
     if (needs_mask != (mask != nullptr)) return SDPA_ERR_NULL_POINTER;
+    if (mask_kind == SDPA_MASK_SLIDING) return SDPA_ERR_INVALID_ARG;   // needs a window: sdpa_forward_window
     if (path == SDPA_PATH_NONE) return SDPA_OK;
-    // this entry point covers the fp16 / bf16 decode path only
+    // this entry point covers the fp16 / bf16 decode path of the tensor-core
+    // decode kernel only (not the absorbed-MLA dims, which run on CUDA cores);
+    // everything here is checked before the first CUDA call
     if (path != SDPA_PATH_DECODE || (dtype != SDPA_F16 && dtype != SDPA_BF16)) return SDPA_ERR_INVALID_ARG;
+    if (!decode_mma_supported(dtype, Dqk, Dv)) return SDPA_ERR_INVALID_ARG;
     if (!out || (Lk > 0 && (!q || !k || !v))) return SDPA_ERR_NULL_POINTER;
     auto misaligned = [](const void* ptr) { return ptr && (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
     if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(out)) return SDPA_ERR_MISALIGNED;
     if (mask_kind == SDPA_MASK_ADDITIVE && (reinterpret_cast<uintptr_t>(mask) & 1u) != 0) return SDPA_ERR_MISALIGNED;
 
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SDPA_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return record_cuda_error(e);
     NoallocDevice nd;
     if ((st = noalloc_device(dev, &nd)) != SDPA_OK) return st;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_ptr);
@@ -116,7 +119,14 @@ extern "C" int sdpa_forward_noalloc(const void* q, const void* k, const void* v,
     p.mask_kind = mask_kind;
     p.group = (int)(Hq / Hkv);
     p.splits = 1;
-    if (Lk == 0) return zero_fill_launch(p, dtype, stream) == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+    p.wait_limit_ns = kWaitLimitNs;
+    p.barrier_extra = 0;
+    p.window = 0;
+    p.key_begin = 0;
+    if (Lk == 0) {
+        if ((e = zero_fill_launch(p, dtype, stream)) != cudaSuccess) return record_cuda_error(e);
+        return SDPA_OK;
+    }
 
     DeviceInfo di{};
     di.device = dev;
@@ -140,8 +150,8 @@ extern "C" int sdpa_forward_noalloc(const void* q, const void* k, const void* v,
         counters = reinterpret_cast<int*>(base);
         p.part_o = reinterpret_cast<float*>(base + kCounterBytes);
         p.part_lse = reinterpret_cast<float*>(base + kCounterBytes + o_bytes);
-        if (cudaMemsetAsync(counters, 0, c_bytes, stream) != cudaSuccess) return SDPA_ERR_CUDA;
+        if ((e = cudaMemsetAsync(counters, 0, c_bytes, stream)) != cudaSuccess) return record_cuda_error(e);
     }
-    if (decode_mma_launch(p, dtype, plan, counters, stream) != cudaSuccess) return SDPA_ERR_CUDA;
+    if ((e = decode_mma_launch(p, dtype, plan, counters, stream)) != cudaSuccess) return record_cuda_error(e);
     return SDPA_OK;
 }

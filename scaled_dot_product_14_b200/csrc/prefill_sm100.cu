@@ -116,6 +116,27 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&o)[16]) {
 }
 
 
+// Key tiles [t0, t0 + n) of `bn` keys that query rows [r_first, r_last] need:
+// causal and sliding-window masks end at the last row's own (bottom-right
+// aligned) key; a sliding window starts at the first row's window.  Tiles
+// outside that range are never loaded.
+template <int MASK>
+__device__ __forceinline__ void key_tiles(const AttnParams& p, int64_t r_first, int64_t r_last, int bn, int& t0,
+                                          int& n) {
+    int64_t k_end = p.Lk, k_begin = 0;
+    if (MASK == 3 || MASK == 4) {
+        const int64_t last = r_last + p.Lk - p.Lq;
+        k_end = last < 0 ? 0 : (last + 1 < p.Lk ? last + 1 : p.Lk);
+    }
+    if (MASK == 4) {
+        const int64_t first = r_first + p.Lk - p.Lq - p.window + 1;
+        k_begin = first < 0 ? 0 : first;
+    }
+    t0 = (int)(k_begin / bn);
+    const int64_t t_end = (k_end + bn - 1) / bn;
+    n = t_end > t0 ? (int)(t_end - t0) : 0;
+}
+
 // ---------------------------------------------------------------- per-row softmax (shared by the kernels)
 // Thread t of a softmax warpgroup owns query row t of its 128-row tile, which
 // is TMEM lane t.  For a key tile of NK keys it loads that row of S, applies
@@ -132,7 +153,7 @@ struct RowSoftmax {
     float m_ref, l;
     bool row_ok, pos_scale;
     float sc;
-    int64_t Lk, causal_lim, mrow, msm3;
+    int64_t Lk, causal_lim, win_lo, mrow, msm3;
     const T* mask_t;
     const uint8_t* mask_b;
 
@@ -144,6 +165,7 @@ struct RowSoftmax {
         pos_scale = sc > 0.f;
         Lk = p.Lk;
         causal_lim = i + p.Lk - p.Lq;
+        win_lo = causal_lim - p.window + 1;   // sliding window: first visible key
         mrow = b * p.sm[0] + hq * p.sm[1] + i * p.sm[2];
         msm3 = p.sm[3];
         mask_t = reinterpret_cast<const T*>(p.mask);
@@ -188,11 +210,13 @@ struct RowSoftmax {
         tmem_wait_ld();
         loaded();
 
-        // keys of this tile that the row may see: [0, vis) (sequence end, causal limit)
+        // keys of this tile that the row may see: [lo, vis) (sequence end, causal
+        // limit; a sliding window also hides the keys before its start)
         int64_t lim = Lk - kbase;
-        if (MASK == 3) lim = min(lim, causal_lim - kbase + 1);
+        if (MASK == 3 || MASK == 4) lim = min(lim, causal_lim - kbase + 1);
         const int vis = row_ok ? (int)max((int64_t)0, min(lim, (int64_t)NK)) : 0;
-        const bool partial = __any_sync(0xffffffffu, vis < NK);   // some key of the tile is hidden
+        const int lo = (MASK == 4) ? (int)max((int64_t)0, min(win_lo - kbase, (int64_t)NK)) : 0;
+        const bool partial = __any_sync(0xffffffffu, vis < NK || lo > 0);   // some key of the tile is hidden
         // values stay raw where possible and are scaled inside the exponent's FFMA
         float mul = sc;
         if (MASK == 1 || MASK == 2 || !pos_scale) {
@@ -202,14 +226,14 @@ struct RowSoftmax {
 #pragma unroll
             for (int c = 0; c < NK; ++c) {
                 float x = __uint_as_float(sr[c]) * sc;
-                bool keep = c < vis;
+                bool keep = c < vis && c >= lo;
                 if (MASK == 1 && keep) x += Elem<T>::to_float(mt_row[(int64_t)c * msm3]) * log2e;
                 if (MASK == 2 && keep) keep = mb_row[(int64_t)c * msm3] != 0;
                 sr[c] = __float_as_uint(keep ? x : -INFINITY);
             }
         } else if (partial) {
 #pragma unroll
-            for (int c = 0; c < NK; ++c) sr[c] = (c < vis) ? sr[c] : __float_as_uint(-INFINITY);
+            for (int c = 0; c < NK; ++c) sr[c] = (c < vis && c >= lo) ? sr[c] : __float_as_uint(-INFINITY);
         }
         float mx8[8];   // eight independent chains of three-input maxima
 #pragma unroll
@@ -326,13 +350,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t q0 = (int64_t)qt * kBM;
     const int dv0 = half * DVC;   // first value column of this CTA
 
-    // number of key tiles this query tile needs (causal: up to the diagonal)
-    int64_t kv_len = p.Lk;
-    if (MASK == 3) {
-        const int64_t last = q0 + kBM - 1 + p.Lk - p.Lq;   // last key that row q0+127 sees
-        kv_len = last < 0 ? 0 : (last + 1 < p.Lk ? last + 1 : p.Lk);
-    }
-    const int n_tiles = (int)((kv_len + kBN - 1) / kBN);
+    // key tiles this query tile needs (causal: up to the diagonal; sliding
+    // window: from the first row's window start)
+    int t0, n_tiles;
+    key_tiles<MASK>(p, q0, q0 + kBM - 1, kBN, t0, n_tiles);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
@@ -373,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int slot = (seq + C::SHIFT) % NSLOT;
                 if (!wait_phase(bar_empty + slot, ((seq / NSLOT) & 1) ^ 1, kErrWaitSlot)) return false;
                 mbar_arrive_expect_tx(bar_full + slot, kChunk);
-                tma_load(ring + slot * kChunk, map, bar_full + slot, ax, d0, j * kBN, hkv, b);
+                tma_load(ring + slot * kChunk, map, bar_full + slot, ax, d0, (t0 + j) * kBN, hkv, b);
                 ++seq;
                 return true;
             };
@@ -508,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             float alpha;
             bool rescale;
-            rs.tile(tmem + lane_off + buf * kBN, (int64_t)j * kBN, alpha, rescale);
+            rs.tile(tmem + lane_off + buf * kBN, (int64_t)(t0 + j) * kBN, alpha, rescale);
             if (j > 0) {
                 ok = __all_sync(0xffffffffu, wait_phase(bar_o_done, (j - 1) & 1, kErrWaitMma));
                 if (!ok) break;
@@ -605,12 +626,10 @@ __global__ void __launch_bounds__(kThreads2, 1)
     const int hkv = hq / p.group;
     const int64_t q0 = (int64_t)pair * 2 * kBM;   // tile A rows [q0, q0+128), tile B the next 128
 
-    int64_t kv_len = p.Lk;   // keys the pair needs (tile B sees the most under causal masking)
-    if (MASK == 3) {
-        const int64_t last = q0 + 2 * kBM - 1 + p.Lk - p.Lq;
-        kv_len = last < 0 ? 0 : (last + 1 < p.Lk ? last + 1 : p.Lk);
-    }
-    const int n_tiles = (int)((kv_len + kBN - 1) / kBN);
+    // key tiles the pair needs (tile B sees the last keys under causal masking,
+    // tile A the first ones under a sliding window)
+    int t0, n_tiles;
+    key_tiles<MASK>(p, q0, q0 + 2 * kBM - 1, kBN, t0, n_tiles);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
@@ -663,7 +682,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
                     if (!(ok = wait_phase(bar_kempty + st, par, kErrWaitSlot))) break;
                     mbar_arrive_expect_tx(bar_kfull + st, C::NBQ * kChunk);
                     for (int c = 0; c < C::NBQ; ++c)
-                        tma_load(slot0 + c * kChunk, &tmK, bar_kfull + st, tp.k_ax, c * 64, j * kBN, hkv, b);
+                        tma_load(slot0 + c * kChunk, &tmK, bar_kfull + st, tp.k_ax, c * 64, (t0 + j) * kBN, hkv,
+                                 b);
                     if (!(ok = wait_phase(bar_vempty + st, par, kErrWaitSlot))) {
                         // K(j) is in flight: land it before the drain below
                         wait_phase(bar_kfull + st, (j / C::NSTAGE) & 1, kErrWaitTmaLoad);
@@ -671,7 +691,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
                     }
                     mbar_arrive_expect_tx(bar_vfull + st, C::NBV * kChunk);
                     for (int c = 0; c < C::NBV; ++c)
-                        tma_load(slot0 + (C::NBQ + c) * kChunk, &tmV, bar_vfull + st, tp.v_ax, c * 64, j * kBN, hkv,
+                        tma_load(slot0 + (C::NBQ + c) * kChunk, &tmV, bar_vfull + st, tp.v_ax, c * 64, (t0 + j) * kBN,
+                                 hkv,
                                  b);
                 }
                 if (!ok) {
@@ -784,7 +805,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
             bool rescale;
             // After each half of P: O is rescaled (before the first half, once
             // P(j-1) V(j-1) has completed) and the MMA issuer is signalled.
-            rs.tile(s_taddr, (int64_t)j * kBN, alpha, rescale, [&](int h, float a, bool rs_needed) {
+            rs.tile(s_taddr, (int64_t)(t0 + j) * kBN, alpha, rescale, [&](int h, float a, bool rs_needed) {
                 if (h == 0 && j > 0 && __any_sync(0xffffffffu, rs_needed)) {
                     ok = __all_sync(0xffffffffu, wait_phase(bar_o_done + x, (j - 1) & 1, kErrWaitMma));
                     tc_fence_after();
@@ -877,12 +898,10 @@ __global__ void __launch_bounds__(kThreads2, 1)
     const int hkv = hq / p.group;
     const int64_t q0 = (int64_t)pair * 2 * kBM;   // tile A rows [q0, q0+128), tile B the next 128
 
-    int64_t kv_len = p.Lk;   // keys the pair needs (tile B sees the most under causal masking)
-    if (MASK == 3) {
-        const int64_t last = q0 + 2 * kBM - 1 + p.Lk - p.Lq;
-        kv_len = last < 0 ? 0 : (last + 1 < p.Lk ? last + 1 : p.Lk);
-    }
-    const int n_tiles = (int)((kv_len + kBN3 - 1) / kBN3);
+    // key tiles the pair needs (tile B sees the last keys under causal masking,
+    // tile A the first ones under a sliding window)
+    int t0, n_tiles;
+    key_tiles<MASK>(p, q0, q0 + 2 * kBM - 1, kBN3, t0, n_tiles);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
@@ -931,14 +950,16 @@ __global__ void __launch_bounds__(kThreads2, 1)
                     if (!(ok = wait_phase(bar_kempty + st, par, kErrWaitSlot))) break;
                     mbar_arrive_expect_tx(bar_kfull + st, C::NBQ * kChunk3);
                     for (int c = 0; c < C::NBQ; ++c)
-                        tma_load(stage + c * kChunk3, &tmK, bar_kfull + st, tp.k_ax, c * 64, j * kBN3, hkv, b);
+                        tma_load(stage + c * kChunk3, &tmK, bar_kfull + st, tp.k_ax, c * 64, (t0 + j) * kBN3, hkv,
+                                 b);
                     if (!(ok = wait_phase(bar_vempty + st, par, kErrWaitSlot))) {
                         wait_phase(bar_kfull + st, (j / NSTAGE) & 1, kErrWaitTmaLoad);   // K(j) is in flight
                         break;
                     }
                     mbar_arrive_expect_tx(bar_vfull + st, C::NBV * kChunk3);
                     for (int c = 0; c < C::NBV; ++c)
-                        tma_load(stage + (C::NBQ + c) * kChunk3, &tmV, bar_vfull + st, tp.v_ax, c * 64, j * kBN3,
+                        tma_load(stage + (C::NBQ + c) * kChunk3, &tmV, bar_vfull + st, tp.v_ax, c * 64,
+                                 (t0 + j) * kBN3,
                                  hkv, b);
                 }
                 if (!ok) {
@@ -1050,7 +1071,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
                 tc_fence_before();
                 mbar_arrive(bar_p_full + x);
             };
-            rs.tile(s_taddr, p_taddr, (int64_t)j * kBN3, alpha, rescale, loaded, before_store, after_store);
+            rs.tile(s_taddr, p_taddr, (int64_t)(t0 + j) * kBN3, alpha, rescale, loaded, before_store, after_store);
         }
         if (ok && n_tiles > 0)
             ok = __all_sync(0xffffffffu, wait_phase(bar_pv + x, (uint32_t)(n_tiles - 1) & 1, kErrWaitMma));
@@ -1138,6 +1159,7 @@ cudaError_t launch_one(const TcParams& tp, const CUtensorMap& mq, const CUtensor
         case 1: return launch_kernel(prefill_tc_kernel<T, DQK, DVC, NSLOT, SPLIT, 1>, tp, mq, mk, mv, plan, stream);
         case 2: return launch_kernel(prefill_tc_kernel<T, DQK, DVC, NSLOT, SPLIT, 2>, tp, mq, mk, mv, plan, stream);
         case 3: return launch_kernel(prefill_tc_kernel<T, DQK, DVC, NSLOT, SPLIT, 3>, tp, mq, mk, mv, plan, stream);
+        case 4: return launch_kernel(prefill_tc_kernel<T, DQK, DVC, NSLOT, SPLIT, 4>, tp, mq, mk, mv, plan, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -1164,6 +1186,7 @@ cudaError_t launch_two(const TcParams& tp, const CUtensorMap& mq, const CUtensor
         case 1: return launch_split_regs(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 1>, tp, mq, mk, mv, plan, stream);
         case 2: return launch_split_regs(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 2>, tp, mq, mk, mv, plan, stream);
         case 3: return launch_split_regs(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 3>, tp, mq, mk, mv, plan, stream);
+        case 4: return launch_split_regs(prefill_tc2_kernel<T, DQK, DVC, NSLOT, 4>, tp, mq, mk, mv, plan, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -1176,6 +1199,7 @@ cudaError_t launch_three(const TcParams& tp, const CUtensorMap& mq, const CUtens
         case 1: return launch_split_regs(prefill_tc3_kernel<T, DQK, DVC, NSTAGE, 1>, tp, mq, mk, mv, plan, stream);
         case 2: return launch_split_regs(prefill_tc3_kernel<T, DQK, DVC, NSTAGE, 2>, tp, mq, mk, mv, plan, stream);
         case 3: return launch_split_regs(prefill_tc3_kernel<T, DQK, DVC, NSTAGE, 3>, tp, mq, mk, mv, plan, stream);
+        case 4: return launch_split_regs(prefill_tc3_kernel<T, DQK, DVC, NSTAGE, 4>, tp, mq, mk, mv, plan, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -1204,7 +1228,6 @@ cudaError_t launch_typed(const TcParams& tp, const CUtensorMap& mq, const CUtens
 
 bool prefill_tc_supported(int dtype, int64_t Dqk, int64_t Dv, const AttnParams& p) {
     (void)p;
-    if (getenv("SDPA_DISABLE_TCGEN05")) return false;
     return (dtype == 1 || dtype == 2) && pick(Dqk, Dv).split != 0;
 }
 

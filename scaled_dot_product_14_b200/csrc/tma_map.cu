@@ -25,16 +25,104 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+// Encoded maps are cached by everything that determines them (the kind of
+// map, base address, dtype, sizes, strides and box rows), so a call repeated
+// on the same tensors does not encode again.  A small table with round-robin
+// replacement; encoding is a host-only computation, so a miss costs only time.
+struct MapKey {
+    int kind, dtype, box_rows;
+    const void* base;
+    int64_t D, L, H, B, st[3];
+    bool operator==(const MapKey& o) const {
+        return kind == o.kind && dtype == o.dtype && box_rows == o.box_rows && base == o.base && D == o.D &&
+               L == o.L && H == o.H && B == o.B && st[0] == o.st[0] && st[1] == o.st[1] && st[2] == o.st[2];
+    }
+};
+struct MapEntry {
+    MapKey key;
+    CUtensorMap map;
+    MapAxes ax;
+    bool used = false;
+};
+constexpr int kMapCache = 64;
+std::mutex g_map_mu;
+MapEntry g_maps[kMapCache];
+int g_map_next = 0;
+
+MapKey map_key(int kind, const void* base, int dtype, int64_t D, int64_t L, int64_t H, int64_t B,
+               const int64_t* st, int box_rows) {
+    MapKey k{};
+    k.kind = kind;
+    k.dtype = dtype;
+    k.box_rows = box_rows;
+    k.base = base;
+    k.D = D;
+    k.L = L;
+    k.H = H;
+    k.B = B;
+    k.st[0] = st[0];
+    k.st[1] = st[1];
+    k.st[2] = st[2];
+    return k;
+}
+
+bool cache_find(const MapKey& k, CUtensorMap* map, MapAxes* ax) {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    for (auto& e : g_maps)
+        if (e.used && e.key == k) {
+            *map = e.map;
+            *ax = e.ax;
+            return true;
+        }
+    return false;
+}
+
+void cache_put(const MapKey& k, const CUtensorMap& map, const MapAxes& ax) {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    MapEntry& e = g_maps[g_map_next];
+    g_map_next = (g_map_next + 1) % kMapCache;
+    e.key = k;
+    e.map = map;
+    e.ax = ax;
+    e.used = true;
+}
+
+bool encode_tiled(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L, int64_t H,
+                  int64_t B, const int64_t* st, int box_rows);
+bool encode_rows(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L, int64_t H,
+                 int64_t B, const int64_t* st, int box_rows);
+
 }  // namespace
+
+bool make_tensor_map(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L, int64_t H,
+                     int64_t B, const int64_t* st, int box_rows) {
+    const MapKey k = map_key(0, base, dtype, D, L, H, B, st, box_rows);
+    if (cache_find(k, map, ax)) return true;
+    if (!encode_tiled(map, ax, base, dtype, D, L, H, B, st, box_rows)) return false;
+    cache_put(k, *map, *ax);
+    return true;
+}
+
+bool make_tensor_map_rows(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L,
+                          int64_t H, int64_t B, const int64_t* st, int box_rows) {
+    const MapKey k = map_key(1, base, dtype, D, L, H, B, st, box_rows);
+    if (cache_find(k, map, ax)) return true;
+    if (!encode_rows(map, ax, base, dtype, D, L, H, B, st, box_rows)) return false;
+    cache_put(k, *map, *ax);
+    return true;
+}
+
+namespace {
 
 // A 4-D tiled map (d, then the sequence / head / batch axes in increasing
 // stride order; an axis of extent 1 or stride 0 is pinned to coordinate 0),
-// 128-byte swizzle, box = 64 elements x box_rows rows, zero fill out of bounds.
-bool make_tensor_map(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L, int64_t H,
-              int64_t B, const int64_t* st, int box_rows) {
+// 128-byte swizzle, box = 128 bytes of d (64 16-bit or 32 fp32 elements) x
+// box_rows rows, zero fill out of bounds.
+bool encode_tiled(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L, int64_t H,
+                  int64_t B, const int64_t* st, int box_rows) {
     auto fn = encode_fn();
     if (!fn) return false;
-    const int64_t esz = 2;
+    const int64_t esz = dtype == 0 ? 4 : 2;
     struct Axis {
         int which;   // 0 = l, 1 = h, 2 = b
         int64_t ext, stride;
@@ -66,12 +154,13 @@ bool make_tensor_map(CUtensorMap* map, MapAxes* ax, const void* base, int dtype,
         gstride[x] = (cuuint64_t)axes[x].stride;
         pos[axes[x].which] = (axes[x].ext > 1 || axes[x].which == 0) ? x + 1 : 0;
     }
-    cuuint32_t box[4] = {64, 1, 1, 1};
+    cuuint32_t box[4] = {(cuuint32_t)(128 / esz), 1, 1, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     for (int x = 0; x < 3; ++x)
         if (axes[x].which == 0) box[x + 1] = (cuuint32_t)box_rows;
-    const CUtensorMapDataType dt =
-        dtype == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const CUtensorMapDataType dt = dtype == 0   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : dtype == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUresult r = fn(map, dt, 4, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -87,10 +176,10 @@ bool make_tensor_map(CUtensorMap* map, MapAxes* ax, const void* base, int dtype,
 // or zero-stride axis is pinned to coordinate 0).  D must be a multiple of 64,
 // so every chunk lies inside its row.  Shared memory receives the box chunk by
 // chunk: [chunk][row][64 elements], the layout of D / 64 separate boxes.
-bool make_tensor_map_rows(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L,
-                          int64_t H, int64_t B, const int64_t* st, int box_rows) {
+bool encode_rows(CUtensorMap* map, MapAxes* ax, const void* base, int dtype, int64_t D, int64_t L, int64_t H,
+                 int64_t B, const int64_t* st, int box_rows) {
     auto fn = encode_fn();
-    if (!fn || D % 64 != 0 || D / 64 > 256) return false;
+    if (!fn || dtype == 0 || D % 64 != 0 || D / 64 > 256) return false;   // 16-bit elements only
     const int64_t esz = 2;
     int64_t span = D * esz;
     const int64_t ext[3] = {L, H, B}, str[3] = {st[2] * esz, st[1] * esz, st[0] * esz};
@@ -122,4 +211,5 @@ bool make_tensor_map_rows(CUtensorMap* map, MapAxes* ax, const void* base, int d
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+}  // namespace
 }  // namespace sdpa

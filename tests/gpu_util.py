@@ -51,6 +51,10 @@ class GpuCase:
         c = self.c
         out_ptr = self.out_buf.data_ptr() + self.pad * self.out_buf.element_size()
         s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+        if c.mask_kind == I.MASK_SLIDING:
+            return S.sdpa_forward_window(self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(), out_ptr,
+                                         c.B, c.Hq, c.Hkv, c.Lq, c.Lk, c.Dqk, c.Dv, c.all_strides16, c.scale,
+                                         c.window, c.dtype, s)
         return S.sdpa_forward(self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(), out_ptr,
                               c.B, c.Hq, c.Hkv, c.Lq, c.Lk, c.Dqk, c.Dv, c.all_strides16, c.scale, c.mask_kind,
                               None if self.mask is None else self.mask.data_ptr(),
@@ -72,7 +76,7 @@ class GpuCase:
 def oracle_rows(c: I.Case, rows=None):
     return oracle.sdpa_rows(c.q, c.k, c.v, B=c.B, Hq=c.Hq, Hkv=c.Hkv, Lq=c.Lq, Lk=c.Lk, Dqk=c.Dqk, Dv=c.Dv,
                             strides=c.strides, scale=c.scale, dtype=c.dtype, mask_kind=c.mask_kind, mask=c.mask,
-                            mask_strides=c.mask_strides, rows=rows)
+                            mask_strides=c.mask_strides, rows=rows, window=c.window)
 
 
 def compare(c: I.Case, got: np.ndarray, rows=None, label=""):

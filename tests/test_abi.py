@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version(lib):
-    assert S.sdpa_abi_version() == 1
+    assert S.sdpa_abi_version() == 2
 
 
 def strides16(layout, B, Hq, Hkv, Lq, Lk, Dqk, Dv):
@@ -69,7 +69,7 @@ def test_invalid_arguments(lib):
     assert sup(Hkv=0, Hq=0)[0] == 1
     assert sup(B=-1)[0] == 1
     assert sup(dtype=3)[0] == 1
-    assert sup(mask_kind=4)[0] == 1
+    assert sup(mask_kind=5)[0] == 1
     assert sup(mask_kind=S.SDPA_MASK_ADDITIVE, mask_strides=None)[0] == 1
 
 
@@ -131,3 +131,45 @@ def test_package_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(S, "_lib", None)
     with pytest.raises(RuntimeError, match="no fallback"):
         S.lib()
+
+
+def test_debug_hooks_validate_their_arguments(lib):
+    assert S.sdpa_debug_set(S.SDPA_DEBUG_WAIT_LIMIT_NS, 0) == 0
+    assert S.sdpa_debug_set(S.SDPA_DEBUG_DECODE_BARRIER_EXTRA, 0) == 0
+    assert S.sdpa_debug_set(S.SDPA_DEBUG_DECODE_BARRIER_EXTRA, -1) == 1
+    assert S.sdpa_debug_set(S.SDPA_DEBUG_DECODE_BARRIER_EXTRA, 5000) == 1
+    assert S.sdpa_debug_set(S.SDPA_DEBUG_FAIL_ALLOCS, -3) == 1
+    assert S.sdpa_debug_set(S.SDPA_DEBUG_FAIL_ALLOCS, 0) == 0
+    assert S.sdpa_debug_set(77, 1) == 1
+    assert S.sdpa_workspace_bytes() >= 0
+
+
+def _noalloc(B=1, Hq=4, Hkv=1, Lq=1, Lk=64, Dqk=40, Dv=32, dtype=2, ptr=4096):
+    st = strides16("bhld", B, Hq, Hkv, Lq, Lk, Dqk, Dv)
+    return S.sdpa_forward_noalloc(ptr, ptr, ptr, ptr, B, Hq, Hkv, Lq, Lk, Dqk, Dv, st, Dqk ** -0.5, 0, None, None,
+                                  dtype, None)
+
+
+def test_noalloc_rejects_uncovered_cases_before_any_cuda_call(lib):
+    """sdpa_forward_noalloc decides every argument status on the host before it
+    touches CUDA, so these run without a GPU: the absorbed-MLA dims (40, 32),
+    which have no tensor-core decode kernel, are refused (once they reached the
+    split planner with an empty shape), as are fp32, prefill lengths and null
+    or misaligned pointers."""
+    assert _noalloc(Dqk=40, Dv=32, dtype=2) == 1
+    assert _noalloc(Dqk=40, Dv=32, dtype=1) == 1
+    assert _noalloc(Dqk=256, Dv=256, dtype=0) == 1
+    assert _noalloc(Dqk=256, Dv=256, Lq=9, Lk=9) == 1
+    assert _noalloc(Dqk=100, Dv=100) == 2
+    assert _noalloc(Dqk=256, Dv=256, ptr=0) == 9
+    assert _noalloc(Dqk=256, Dv=256, ptr=4096 + 2) == 4
+    assert _noalloc(Dqk=256, Dv=256, B=0) == 0
+
+
+def test_sliding_window_kind_is_validated_on_the_host(lib):
+    assert sup(mask_kind=S.SDPA_MASK_SLIDING) == (0, S.SDPA_PATH_DECODE)
+    assert sup(mask_kind=S.SDPA_MASK_SLIDING, Lq=100, Lk=100) == (0, S.SDPA_PATH_PREFILL)
+    assert sup(mask_kind=5)[0] == 1
+    st = strides16("bhld", 1, 4, 2, 16, 16, 64, 64)
+    # window < 1 is refused before any CUDA call
+    assert S.sdpa_forward_window(4096, 4096, 4096, 4096, 1, 4, 2, 16, 16, 64, 64, st, 0.125, 0, 2, None) == 1

@@ -123,16 +123,13 @@ def test_prefill_d512_causal_4096():
 @pytest.mark.parametrize("dtype,mask", [(I.BF16, "none"), (I.F16, "none"), (I.BF16, "bool")])
 def test_prefill_d72_8192(dtype, mask):
     c = I.make_case(1003, 1, 16, 16, 8192, 8192, 72, dtype=dtype, mask=mask, layout="blhd", p_keep=0.9)
-    rows = I.sample_rows(1003, 1, 16, 8192, 64)
+    rows = I.sample_rows(1003, 1, 16, 8192, 256)
     run_and_check(c, rows=rows, label=f"prefill d72 {dtype} {mask}")
 
 
 # ---------------------------------------------------------------- the coverage sweep
 def _sweep_case(D, Dv, dtype, mask, L, seed, B=2):
-    # at the largest size the additive mask is broadcast over the batch ([1,1,L,L]) to bound host memory
-    m = {"additive": "additive" if L < 16384 else "additive_bcast", "bool": "bool", "causal": "causal",
-         "none": "none"}[mask]
-    return I.make_case(seed, B, 32, 8, L, L, D, Dv, dtype=dtype, mask=m)
+    return I.make_case(seed, B, 32, 8, L, L, D, Dv, dtype=dtype, mask=mask)
 
 
 @pytest.mark.parametrize("D,Dv", DIMS)
@@ -152,14 +149,41 @@ def test_sweep_L2048_sampled(D, Dv, dtype, mask):
     run_and_check(c, rows=rows, label=f"sweep L=2048 D={D} dt={dtype} {mask}")
 
 
-@pytest.mark.parametrize("D,Dv", DIMS)
-@pytest.mark.parametrize("dtype", DTYPES)
-def test_sweep_L16384_sampled(D, Dv, dtype):
-    # one mask per (dim, dtype), cycling, to bound the run time of the largest size
-    mask = MASKS[(DIMS.index((D, Dv)) + DTYPES.index(dtype)) % 4]
-    c = _sweep_case(D, Dv, dtype, mask, 16384, 1006, B=1)
-    rows = I.sample_rows(1006, 1, 32, 16384, 24)
-    run_and_check(c, rows=rows, label=f"sweep L=16384 D={D} dt={dtype} {mask}")
+_L16K_MASKS = {}
+
+
+def _l16k_masks(dtype):
+    """The configured masks of the L=16384 sweep for one dtype: additive
+    [B,1,Lq,Lk] U(-1,0) and boolean [1,1,Lq,Lk] (p_keep 0.9), each drawn once
+    from its own seeded generator and shared by every head dim (one draw of the
+    1.07 G-element additive mask takes seconds on the host)."""
+    if dtype not in _L16K_MASKS:
+        _L16K_MASKS.clear()
+        L = 16384
+        add = np.random.default_rng(1006 + 50000).uniform(-1.0, 0.0, size=(2, 1, L, L)).astype(np.float32)
+        keep = (np.random.default_rng(1006 + 60000).random((L, L)) < 0.9).astype(np.uint8)
+        _L16K_MASKS[dtype] = (I.to_storage(add.reshape(-1), dtype), keep.reshape(-1))
+    return _L16K_MASKS[dtype]
+
+
+@pytest.mark.parametrize("dtype,D,Dv", [(dt, D, Dv) for dt in DTYPES for (D, Dv) in DIMS])
+def test_sweep_L16384_sampled(dtype, D, Dv):
+    """Every (head dim, dtype, mask) cell of the sweep at L=16384, B=2, Hq=32,
+    Hkv=8, on seeded sampled rows (plus the first and last rows): the same
+    Q/K/V for the four masks, the additive mask [B,1,Lq,Lk] as configured."""
+    import dataclasses
+    L = 16384
+    base = I.make_case(1006, 2, 32, 8, L, L, D, Dv, dtype=dtype, mask="none")
+    add, keep = _l16k_masks(dtype)
+    variants = {
+        "none": base,
+        "causal": dataclasses.replace(base, mask_kind=I.MASK_CAUSAL),
+        "additive": dataclasses.replace(base, mask_kind=I.MASK_ADDITIVE, mask=add, mask_strides=(L * L, 0, L, 1)),
+        "bool": dataclasses.replace(base, mask_kind=I.MASK_BOOL, mask=keep, mask_strides=(0, 0, L, 1)),
+    }
+    rows = I.sample_rows(1006 + D, 2, 32, L, 32)
+    for mask in MASKS:
+        run_and_check(variants[mask], rows=rows, label=f"sweep L=16384 D={D} dt={dtype} {mask}")
 
 
 @pytest.mark.parametrize("D,Dv", DIMS)
@@ -272,17 +296,40 @@ def test_layouts_agree_on_gpu():
     assert np.abs(ga - gb).max() <= 1e-6
 
 
+TF32_DIMS = [(40, 32), (64, 64), (72, 72), (80, 80), (96, 96)]
+
+
 @pytest.mark.parametrize("D,Dv", [(64, 64), (72, 72), (80, 80), (96, 96), (128, 128), (192, 128)])
 @pytest.mark.parametrize("mask", MASKS)
-def test_fp32_tiled_prefill_tiles(D, Dv, mask):
-    """fp32 prefill on the register-tiled kernel (128 group rows per CTA, 64-key
-    tiles): Lq=100 with 4 query heads per KV head puts rows of two heads in one
-    row tile, and Lk=200 leaves a ragged last key tile."""
+def test_fp32_prefill_tiles(D, Dv, mask):
+    """fp32 prefill: the tcgen05 three-term TF32 kernel at head dims up to 96
+    (128-row query tiles, 64-key tiles), the register-tiled FFMA kernel above
+    (128 group rows per CTA, 64-key tiles): Lq=100 with 4 query heads per KV
+    head puts rows of two heads in one FFMA row tile, and Lk=200 leaves a ragged
+    last key tile on both."""
     c = I.make_case(1900 + D, 2, 8, 2, 100, 200, D, Dv, dtype=I.F32, mask=mask, layout="blhd", p_keep=0.7)
     before = S.sdpa_get_counters()
-    run_and_check(c, label=f"fp32 tiled D={D} {mask}")
+    run_and_check(c, label=f"fp32 D={D} {mask}")
     after = S.sdpa_get_counters()
-    assert after["prefill_ffma_launches"] == before["prefill_ffma_launches"] + 1
+    fam = "prefill_tf32_launches" if (D, Dv) in TF32_DIMS else "prefill_ffma_launches"
+    assert after[fam] == before[fam] + 1
+
+
+@pytest.mark.parametrize("D,Dv", TF32_DIMS)
+@pytest.mark.parametrize("mask", MASKS + ["sliding"])
+@pytest.mark.parametrize("Lq,Lk", [(129, 129), (300, 1000), (1000, 300), (2048, 2048)])
+def test_fp32_three_term_tf32_holds_fp32_accuracy(D, Dv, mask, Lq, Lk):
+    """mlxcel issue #1065: TF32 inside an fp32 path must not show up as error;
+    the three-term split keeps max-abs <= 1e-5 against the float64 oracle (far
+    below the 2^-10 fingerprint of plain TF32) over ragged tiles, Lq != Lk and
+    every mask kind; sampled rows at the larger sizes."""
+    c = I.make_case(2600 + D + Lq, 1, 8, 2, Lq, Lk, D, Dv, dtype=I.F32, mask=mask, p_keep=0.7, window=150)
+    before = S.sdpa_get_counters()
+    rows = None if Lq * Lk <= 300_000 else I.sample_rows(2600 + D, 1, 8, Lq, 96)
+    (mx, _), _ = run_and_check(c, rows=rows, label=f"tf32x3 D={D} {mask} {Lq}x{Lk}")
+    after = S.sdpa_get_counters()
+    assert after["prefill_tf32_launches"] == before["prefill_tf32_launches"] + 1
+    assert mx <= 1e-5 < 2.0 ** -10
 
 
 def test_fp32_keeps_fp32_precision():
@@ -307,3 +354,65 @@ def test_repeat_calls_are_deterministic():
 def test_counters_invariant():
     c = S.sdpa_get_counters()
     assert c["calls"] == c["prefill_calls"] + c["decode_calls"] + c["empty_calls"] + c["rejected_calls"]
+
+
+# ---------------------------------------------------------------- sliding window (NEXT: local attention)
+# Gemma 4's sliding layers (MLX issue #3885, "Current routing": n_q=32, n_kv=16,
+# d=256) next to its global ones; the rule is the reading documented with the
+# oracle: with own = i + Lk - Lq, key j is visible iff own - W < j <= own.
+@pytest.mark.parametrize("D,Dv", DIMS)
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("W", [1, 77, 300])
+def test_sliding_window_prefill(D, Dv, dtype, W):
+    """Lq < Lk with ragged tiles: windows narrower than one key tile, spanning
+    a few tiles, and wider than most rows' history; every row checked."""
+    c = I.make_case(2100 + W, 1, 8, 2, 333, 517, D, Dv, dtype=dtype, mask="sliding", window=W)
+    assert path_of(c) == S.SDPA_PATH_PREFILL
+    run_and_check(c, label=f"sliding W={W} D={D} dt={dtype}")
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("D,Dv", [(72, 72), (128, 128), (256, 256), (512, 512)])
+def test_sliding_window_long_prefill_skips_tiles(D, Dv, dtype):
+    """L = 4096 with a 256-key window: most key tiles of a query tile lie
+    outside every row's window and are never loaded; sampled rows, including
+    the first rows (whose windows are cut at key 0)."""
+    c = I.make_case(2200, 1, 8, 4, 4096, 4096, D, Dv, dtype=dtype, mask="sliding", window=256)
+    rows = np.concatenate([I.sample_rows(2200, 1, 8, 4096, 48),
+                           np.array([[0, 3, i] for i in (1, 2, 255, 256, 257)])])
+    run_and_check(c, rows=np.unique(rows, axis=0), label=f"sliding long D={D} dt={dtype}")
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("Lq", [1, 4, 8])
+@pytest.mark.parametrize("W", [1, 100, 1024, 5000])
+def test_sliding_window_decode_gemma4_shape(dtype, Lq, W):
+    """The decode path on the sliding-layer shape (32 q / 16 kv heads, d=256),
+    kL=4096: the splits divide the window's keys only."""
+    c = I.make_case(2300 + W, 1, 32, 16, Lq, 4096, 256, dtype=dtype, mask="sliding", window=W)
+    assert path_of(c) == S.SDPA_PATH_DECODE
+    run_and_check(c, label=f"sliding decode W={W} Lq={Lq} dt={dtype}")
+
+
+@pytest.mark.parametrize("D,Dv", DIMS)
+def test_sliding_window_equals_causal_when_it_covers_every_key(D, Dv):
+    import dataclasses
+    c = I.make_case(2400, 2, 8, 2, 129, 129, D, Dv, dtype=I.BF16, mask="sliding", window=129)
+    (_, _), a = run_and_check(c, label="window = Lk")
+    (_, _), b = run_and_check(dataclasses.replace(c, mask_kind=I.MASK_CAUSAL, window=0), label="causal")
+    assert np.abs(a - b).max() <= 1e-6
+
+
+def test_sliding_window_abi_rules():
+    c = I.make_case(2500, 1, 4, 2, 16, 16, 64, dtype=I.BF16)
+    g = GpuCase(c)
+    out = g.out_buf.data_ptr() + g.pad * g.out_buf.element_size()
+    args = (g.q.data_ptr(), g.k.data_ptr(), g.v.data_ptr(), out, c.B, c.Hq, c.Hkv, c.Lq, c.Lk, c.Dqk, c.Dv,
+            c.all_strides16, c.scale)
+    s = torch.cuda.current_stream().cuda_stream
+    assert S.sdpa_forward_window(*args, 0, c.dtype, s) == 1                       # window >= 1
+    assert S.sdpa_forward(*args, S.SDPA_MASK_SLIDING, None, None, c.dtype, s) == 1  # needs the window entry
+    assert S.sdpa_supported(c.B, c.Hq, c.Hkv, c.Lq, c.Lk, c.Dqk, c.Dv, c.all_strides16, S.SDPA_MASK_SLIDING,
+                            None, c.dtype) == (0, S.SDPA_PATH_PREFILL)
+    assert S.sdpa_forward_window(*args, 5, c.dtype, s) == 0
+    torch.cuda.synchronize()

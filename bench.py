@@ -652,7 +652,8 @@ def mla_leg(S, stream, peaks, rank, args):
         res.append({"workload": w["name"], "dtype": dt, "us_per_call": round(us, 3),
                     "algorithmic_bytes": nbytes, "mask_bytes": e * c.Lk, "achieved_gbs": round(gbs, 1),
                     "peak_gbs": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4),
-                    "bound": "latency (0.3-0.7 MB per call: memory round trips and two launches, not bandwidth)", "launches_per_call": S.sdpa_last_launch_count(),
+                    "bound": "latency (0.3-0.7 MB per call: memory round trips, not bandwidth)",
+                    "launches_per_call": S.sdpa_last_launch_count(),
                     "iters": n, "timing": "median", "l2": "flushed between timed launches"})
         del t, out
     del flush

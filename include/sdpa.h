@@ -100,7 +100,8 @@ typedef enum {
     SDPA_PATH_PREFILL = 1,  /* Lq > 8: tiled flash kernel (tcgen05 kind::f16 for fp16/bf16; for fp32
                                tcgen05 kind::tf32 with a three-term hi/lo split at head dims
                                (40,32), 64, 72, 80, 96, FFMA at the others) */
-    SDPA_PATH_DECODE = 2    /* Lq <= 8: split-K kernel plus log-sum-exp combine */
+    SDPA_PATH_DECODE = 2    /* Lq <= 8: split-K kernel with the log-sum-exp merge of its
+                               splits in the same launch */
 } sdpa_path;
 
 /*
@@ -227,7 +228,8 @@ typedef struct {
     uint64_t prefill_ffma_launches;     /* fp32 prefill on CUDA cores */
     uint64_t decode_mma_launches;       /* fp16/bf16 split-K decode */
     uint64_t decode_ffma_launches;      /* fp32 split-K decode */
-    uint64_t combine_launches;          /* log-sum-exp combine of split-K partials */
+    uint64_t combine_launches;          /* separate combine launches: always 0 (every split kernel
+                                           merges its partials in the same launch) */
     uint64_t prefill_tf32_launches;     /* fp32 prefill on tcgen05 kind::tf32, three-term split */
 } sdpa_counters;
 
@@ -236,7 +238,8 @@ void sdpa_reset_counters(void);
 
 /*
  * Kernel launches the most recent successful sdpa_forward on this thread
- * made (1 or 2).  Lets a caller count launches without a profiler.
+ * made (1, or 0 for an empty problem).  Lets a caller count launches without
+ * a profiler.
  */
 int sdpa_last_launch_count(void);
 

@@ -379,9 +379,14 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, int64_t
             const size_t l_bytes = (size_t)rows * p.splits * sizeof(float);
             void* ws = nullptr;
             if ((st = workspace(dev.device, stream, o_bytes + l_bytes + 256, &ws)) != SDPA_OK) return reject(st);
-            if (mma && (st = counter_region(dev.device, stream, (int64_t)plan.grid.x, plan.split_lo,
-                                            plan.split_extra, decode_mma_counters(p, plan), &counters)) != SDPA_OK)
+            // tensor-core decode: a split barrier; CUDA-core decode: the last split
+            // of a tile merges it (both in the one launch)
+            const int64_t shape_key = mma ? (int64_t)plan.grid.x : -(int64_t)plan.grid.x * plan.grid.y * plan.grid.z;
+            const size_t n_cnt = mma ? decode_mma_counters(p, plan) : ffma_counters(plan);
+            if ((st = counter_region(dev.device, stream, shape_key, plan.split_lo, mma ? plan.split_extra : plan.splits,
+                                     n_cnt, &counters)) != SDPA_OK)
                 return reject(st);
+            if (!mma) p.counters = counters;
             p.part_o = reinterpret_cast<float*>(ws);
             p.part_lse = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + ((o_bytes + 255) / 256) * 256);
         }
@@ -392,13 +397,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, int64_t
         if (e != cudaSuccess) return cuda_fail(e);
         (mma ? c_dmma : c_dffma).fetch_add(1, std::memory_order_relaxed);
         launches = 1;
-        if (p.splits > 1 && !mma) {   // the mma decode kernel merges its splits itself
-            if ((e = timed(SDPA_KERNEL_COMBINE, stream, [&] { return combine_launch(p, dtype, stream); })) !=
-                cudaSuccess)
-                return cuda_fail(e);
-            c_combine.fetch_add(1, std::memory_order_relaxed);
-            launches = 2;
-        }
+
         c_decode.fetch_add(1, std::memory_order_relaxed);
     } else {
         // fp16 / bf16 on tcgen05 kind::f16; fp32 on tcgen05 kind::tf32 with the

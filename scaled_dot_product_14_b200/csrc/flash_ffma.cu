@@ -207,19 +207,57 @@ __global__ void __launch_bounds__(kThreads) flash_ffma_kernel(const AttnParams p
     l += __shfl_xor_sync(0xffffffffu, l, 1);
     l += __shfl_xor_sync(0xffffffffu, l, 2);
     l += __shfl_xor_sync(0xffffffffu, l, 4);
-    if (!row_ok) return;
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    T* og = reinterpret_cast<T*>(p.out) + b * p.so[0] + hq * p.so[1] + qi * p.so[2];
     if (p.splits == 1) {
-        T* og = reinterpret_cast<T*>(p.out) + b * p.so[0] + hq * p.so[1] + qi * p.so[2];
+        if (row_ok)
 #pragma unroll
-        for (int u = 0; u < DV / 8; ++u) og[c8 + 8 * u] = Elem<T>::from_float(o[u] * inv);
-    } else {
-        const int64_t row = ((int64_t)b * p.Hq + hq) * p.Lq + qi;
-        float* po = p.part_o + (row * p.splits + split) * DV;
+            for (int u = 0; u < DV / 8; ++u) og[c8 + 8 * u] = Elem<T>::from_float(o[u] * inv);
+        return;
+    }
+    const int NS = p.splits;
+    const int64_t row = ((int64_t)b * p.Hq + hq) * p.Lq + qi;
+    if (row_ok) {
+        float* po = p.part_o + (row * NS + split) * DV;
 #pragma unroll
         for (int u = 0; u < DV / 8; ++u) po[c8 + 8 * u] = o[u] * inv;
-        if (c8 == 0) p.part_lse[row * p.splits + split] = (l > 0.f) ? m + log2f(l) : -INFINITY;
+        if (c8 == 0) p.part_lse[row * NS + split] = (l > 0.f) ? m + log2f(l) : -INFINITY;
     }
+    if (p.counters == nullptr) return;   // (never with splits > 1: the dispatcher always passes counters)
+
+    // The last split of this (row tile, KV head, batch) to finish merges the
+    // tile's rows over all splits; no CTA waits for another, so the grid may
+    // run in waves.  Every call adds exactly NS to the tile's 64-bit counter
+    // (counters are kept per launch shape), so the last arrival is the one
+    // that brings it to a multiple of NS.
+    __shared__ int s_last;
+    __syncthreads();   // every thread's partial stores precede thread 0's release below
+    if (tid == 0) {
+        unsigned long long* ctr = reinterpret_cast<unsigned long long*>(p.counters) +
+                                  ((int64_t)blockIdx.z / NS * gridDim.y + hkv) * gridDim.x + blockIdx.x;
+        unsigned long long old;
+        asm volatile("atom.add.acq_rel.gpu.global.u64 %0, [%1], 1;" : "=l"(old) : "l"(ctr) : "memory");
+        s_last = ((old + 1) % (unsigned long long)NS) == 0;
+    }
+    __syncthreads();   // thread 0's acquire orders the other splits' partials before these loads
+    if (!s_last || !row_ok) return;
+    const float* pl = p.part_lse + row * NS;
+    float mx = -INFINITY;
+    for (int s2 = 0; s2 < NS; ++s2) mx = fmaxf(mx, __ldcg(pl + s2));
+    float acc[DV / 8], wsum = 0.f;
+#pragma unroll
+    for (int u = 0; u < DV / 8; ++u) acc[u] = 0.f;
+    for (int s2 = 0; s2 < NS; ++s2) {
+        const float ls = __ldcg(pl + s2);
+        const float ws = (mx == -INFINITY || ls == -INFINITY) ? 0.f : exp2f(ls - mx);
+        wsum += ws;
+        const float* ps = p.part_o + (row * NS + s2) * DV;
+#pragma unroll
+        for (int u = 0; u < DV / 8; ++u) acc[u] = fmaf(ws, __ldcg(ps + c8 + 8 * u), acc[u]);
+    }
+    const float winv = (wsum > 0.f) ? 1.f / wsum : 0.f;
+#pragma unroll
+    for (int u = 0; u < DV / 8; ++u) og[c8 + 8 * u] = Elem<T>::from_float(acc[u] * winv);
 }
 
 // ---- register-tiled fp32 prefill ------------------------------------------
@@ -659,6 +697,10 @@ LaunchPlan ffma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev, bool
     plan.keys_per_split = kps;
     plan.variant = 0;
     return plan;
+}
+
+size_t ffma_counters(const LaunchPlan& plan) {
+    return (size_t)plan.grid.x * plan.grid.y * (plan.grid.z / (plan.splits > 0 ? plan.splits : 1)) * 2;
 }
 
 cudaError_t ffma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, cudaStream_t stream) {

@@ -47,6 +47,10 @@ struct AttnParams {
     int64_t keys_per_split;
     float* part_o;        // [rows][splits][Dv]   rows = B*Hq*Lq, row = (b*Hq + h)*Lq + i
     float* part_lse;      // [rows][splits]       log2-domain log-sum-exp, -inf = no key
+    // CUDA-core split-key decode: one 64-bit arrival counter per (row tile, KV
+    // head, batch); with it the last split to finish merges the tile in the
+    // same launch (nullptr: a separate combine launch merges)
+    int* counters;
     // bounded in-kernel waits of the decode kernel give up after this many
     // nanoseconds (the dispatcher passes about 2 s unless a test hook asks for less)
     uint64_t wait_limit_ns;
@@ -105,6 +109,8 @@ bool make_tensor_map_rows(CUtensorMap* map, MapAxes* ax, const void* base, int d
 // ---- fp32 (and generic) flash kernel on CUDA cores: flash_ffma.cu
 bool ffma_supported(int dtype, int64_t Dqk, int64_t Dv);
 LaunchPlan ffma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev, bool split_keys);
+// ints of counter space the split-key plan's in-launch merge needs
+size_t ffma_counters(const LaunchPlan& plan);
 cudaError_t ffma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, cudaStream_t stream);
 
 // ---- fp16/bf16 split-K decode (TMA + mma.sync, combine fused): decode_mma.cu
@@ -118,8 +124,7 @@ size_t decode_mma_counters(const AttnParams& p, const LaunchPlan& plan);
 cudaError_t decode_mma_launch(const AttnParams& p, int dtype, const LaunchPlan& plan, int* counters,
                               cudaStream_t stream);
 
-// ---- log-sum-exp combine of split-K partials + zero fill: combine.cu
-cudaError_t combine_launch(const AttnParams& p, int dtype, cudaStream_t stream);
+// ---- zero fill of the output of a problem with no keys: combine.cu
 cudaError_t zero_fill_launch(const AttnParams& p, int dtype, cudaStream_t stream);
 
 // ---- fp16/bf16 prefill on tcgen05 / TMEM / TMA: prefill_sm100.cu

@@ -156,6 +156,14 @@ struct RowSoftmax {
     int64_t Lk, causal_lim, win_lo, mrow, msm3;
     const T* mask_t;
     const uint8_t* mask_b;
+    // The row's mask values of the next key tile, loaded as 16-byte vectors
+    // while the current tile is processed (additive: NK 16-bit values; boolean:
+    // NK bytes).  Used when the row's tile is contiguous (key stride 1),
+    // 16-byte aligned and inside the row (not the ragged last tile); otherwise
+    // the tile's values are read one by one.
+    static constexpr int MV = MASK == 1 ? NK * 2 / 16 : MASK == 2 ? NK / 16 : 1;
+    uint4 mvec[MV];
+    int64_t mvec_kbase;   // the tile mvec holds, or -1
 
     __device__ __forceinline__ void init(const AttnParams& p, int64_t b, int64_t hq, int64_t i) {
         m_ref = -INFINITY;
@@ -170,6 +178,23 @@ struct RowSoftmax {
         msm3 = p.sm[3];
         mask_t = reinterpret_cast<const T*>(p.mask);
         mask_b = reinterpret_cast<const uint8_t*>(p.mask);
+        mvec_kbase = -1;
+    }
+
+    // Issue the vector loads of the mask tile at kbase (no-op when the tile
+    // cannot take them: it is then read element by element in tile()).
+    __device__ __forceinline__ void fetch_mask(int64_t kbase) {
+        mvec_kbase = -1;
+        if (MASK != 1 && MASK != 2) return;
+        if (MASK == 1 && NK > 96) return;   // 64 more registers next to 128 scores would spill
+        if (!row_ok || msm3 != 1 || kbase < 0 || kbase + NK > Lk) return;
+        const void* src = MASK == 1 ? static_cast<const void*>(mask_t + mrow + kbase)
+                                    : static_cast<const void*>(mask_b + mrow + kbase);
+        if ((reinterpret_cast<uintptr_t>(src) & 15u) != 0) return;
+        const uint4* v = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+        for (int u = 0; u < MV; ++u) mvec[u] = __ldg(v + u);
+        mvec_kbase = kbase;
     }
 
     // NP pairs: p = 2^(x * mul - m) (MUFU), summed into acc, packed into pr.
@@ -219,17 +244,38 @@ struct RowSoftmax {
         const bool partial = __any_sync(0xffffffffu, vis < NK || lo > 0);   // some key of the tile is hidden
         // values stay raw where possible and are scaled inside the exponent's FFMA
         float mul = sc;
-        if (MASK == 1 || MASK == 2 || !pos_scale) {
+        if (MASK == 1 || MASK == 2) {
             mul = 1.f;
+            // this tile's values: the vectors requested during the previous tile
+            // (or now); they are applied first, and then the next tile's vectors
+            // are requested, so one set is live at a time (an additive mask at
+            // 128-key tiles is read element by element: its 64 registers next to
+            // the 128 scores would spill)
+            if (mvec_kbase != kbase) fetch_mask(kbase);
+            const bool vec = mvec_kbase == kbase;
             const T* mt_row = mask_t + mrow + kbase * msm3;
             const uint8_t* mb_row = mask_b + mrow + kbase * msm3;
 #pragma unroll
             for (int c = 0; c < NK; ++c) {
                 float x = __uint_as_float(sr[c]) * sc;
                 bool keep = c < vis && c >= lo;
-                if (MASK == 1 && keep) x += Elem<T>::to_float(mt_row[(int64_t)c * msm3]) * log2e;
-                if (MASK == 2 && keep) keep = mb_row[(int64_t)c * msm3] != 0;
+                if (MASK == 1 && keep) {
+                    const T mv = vec ? reinterpret_cast<const T*>(mvec)[c] : mt_row[(int64_t)c * msm3];
+                    x += Elem<T>::to_float(mv) * log2e;
+                }
+                if (MASK == 2 && keep) {
+                    const uint8_t mb = vec ? reinterpret_cast<const uint8_t*>(mvec)[c] : mb_row[(int64_t)c * msm3];
+                    keep = mb != 0;
+                }
                 sr[c] = __float_as_uint(keep ? x : -INFINITY);
+            }
+            fetch_mask(kbase + NK);
+        } else if (!pos_scale) {
+            mul = 1.f;
+#pragma unroll
+            for (int c = 0; c < NK; ++c) {
+                const float x = __uint_as_float(sr[c]) * sc;
+                sr[c] = __float_as_uint((c < vis && c >= lo) ? x : -INFINITY);
             }
         } else if (partial) {
 #pragma unroll

@@ -210,7 +210,9 @@ int sdpa_supported(int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk,
 /* Static text for a status code. */
 const char* sdpa_error_string(int status);
 
-/* Text of the last CUDA error seen by this thread's sdpa_forward ("" if none). */
+/* Text of the CUDA error (or failed workspace allocation) of this thread's most
+ * recent sdpa_forward, sdpa_forward_window or sdpa_forward_noalloc call; ""
+ * when that call had none.  Each call clears it on entry. */
 const char* sdpa_last_cuda_error(void);
 
 /*

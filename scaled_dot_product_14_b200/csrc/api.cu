@@ -286,6 +286,8 @@ int record_cuda_error(cudaError_t e) {
     return cuda_fail(e);
 }
 
+void clear_last_cuda_error() { t_last_cuda_error.clear(); }
+
 }  // namespace sdpa
 
 using namespace sdpa;
@@ -310,6 +312,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, int64_t
                  void* stream_ptr) {
     c_calls.fetch_add(1, std::memory_order_relaxed);
     t_last_launches = 0;
+    t_last_cuda_error.clear();
     auto reject = [](int st) {
         c_rejected.fetch_add(1, std::memory_order_relaxed);
         return st;

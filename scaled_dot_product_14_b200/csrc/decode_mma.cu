@@ -50,6 +50,8 @@ constexpr int kMaxSplits = 256;
 __host__ __device__ constexpr int round16(int x) { return (x + 15) / 16 * 16; }
 __host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
+__host__ __device__ constexpr int imin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ constexpr int imax(int a, int b) { return a > b ? a : b; }
 
 // SK keys per ring slot; a slot holds K then V, each as 64-element column chunks
 // of SK rows x 128 bytes (128-byte swizzle).
@@ -70,7 +72,12 @@ struct DecodeCfg {
     static constexpr int MERGE_FLOATS = W * ROWS * MS;
     static constexpr int OFF_ROWS = OFF_BAR + 2 * NSLOT * 8 + 16;
     static constexpr int OFF_COEF = OFF_ROWS + 2 * ROWS * 8;   // [ROWS][W + 1]: merge weights, then lse
-    static constexpr int SMEM = OFF_COEF + ROWS * (W + 1) * 4 + 1024;
+    static constexpr int OFF_MPRE = (OFF_COEF + ROWS * (W + 1) * 4 + 127) / 128 * 128;
+    static constexpr int MPRE = 8192;            // mask values of the CTA's keys, copied up front
+    static constexpr int SMEM = OFF_MPRE + MPRE + 1024;
+    // slots the producer keeps in flight: about 96 KB per SM (a deeper queue
+    // only delays the first slot of every CTA, and every other load behind it)
+    static constexpr int INFLIGHT = imin(imax(98304 / SLOT, 3), NSLOT);
     static constexpr int THREADS = (W + 1) * 32;
     static_assert(MERGE_FLOATS * 4 <= NSLOT * SLOT, "merge area must fit in the ring");
     static_assert(SMEM <= 232448, "shared memory budget");
@@ -122,6 +129,14 @@ __device__ __forceinline__ bool split_barrier(unsigned long long* counter, unsig
     }
 }
 
+// untiled bulk copy global -> this CTA's shared memory, completing on `bar`
+// (16-byte aligned addresses, a multiple of 16 bytes)
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 template <int NT>
 struct MaskFrag {
     float add[NT][4];
@@ -144,6 +159,8 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* bar_empty = bar_full + NSLOT;
     int* s_flag = reinterpret_cast<int*>(bar_empty + NSLOT);
+    uint64_t* bar_mask = bar_empty + NSLOT + 1;   // the mask values copied up front
+    const unsigned char* mpre = smem + C::OFF_MPRE;
     int64_t* row_out = reinterpret_cast<int64_t*>(smem + C::OFF_ROWS);     // [ROWS] output element offset
     int64_t* row_part = row_out + C::ROWS;                                  // [ROWS] partial row index, -1 = none
 
@@ -178,8 +195,9 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     if (tid == 0) {
         for (int s = 0; s < NSLOT; ++s) {
             mbar_init(bar_full + s, 1);
-            mbar_init(bar_empty + s, kNSUB);   // each 16-key sub-block's consumer arrives once
+            mbar_init(bar_empty + s, W);   // every consumer warp arrives once per slot
         }
+        mbar_init(bar_mask, 1);
         fence_barrier_init();
         tma_prefetch_desc(&tmK);   // kernel parameters: safe before the wait below
         tma_prefetch_desc(&tmV);
@@ -206,6 +224,36 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         sl_end = sl_first + nv * (split + 1) / S;
     }
     const int n_slots = sl_end > sl_begin ? (int)(sl_end - sl_begin) : 0;
+    const int n_rows = (int)min((int64_t)C::ROWS, R - row0);   // real query rows of this CTA
+
+    // ---- additive / boolean mask values of this CTA's keys go to shared memory
+    // up front, one bulk copy per distinct mask row issued before the first K/V
+    // slot, when each row's run is contiguous and 16-byte aligned and all of
+    // them fit: loads issued later would queue behind the CTA's K/V stream.
+    // Keys [pre_k0, pre_end) are then read from shared memory (the ragged
+    // last bytes of the run, if any, from global memory).
+    const int64_t esz = p.mask_kind == 1 ? (int64_t)sizeof(T) : 1;
+    auto mask_row = [&](int r) -> int64_t {   // element offset of CTA row r's mask row
+        const int64_t gr = row0 + r;
+        return b * p.sm[0] + (hkv * G + gr / p.Lq) * p.sm[1] + (gr % p.Lq) * p.sm[2];
+    };
+    int64_t pre_k0 = 0, pre_end = 0;
+    int pre_rows = 0;
+    uint32_t pre_pitch = 0;
+    if ((p.mask_kind == 1 || p.mask_kind == 2) && p.sm[3] == 1 && n_slots > 0) {
+        const int64_t k0 = sl_begin * SK, k1 = min(sl_end * SK, p.Lk);
+        const uint32_t nb = (uint32_t)(((k1 - k0) * esz) & ~(int64_t)15);
+        const int rows = (p.sm[1] == 0 && (p.sm[2] == 0 || p.Lq == 1)) ? 1 : n_rows;
+        bool ok = nb > 0 && (int64_t)rows * nb <= C::MPRE;
+        for (int r = 0; r < rows && ok; ++r)
+            ok = ((reinterpret_cast<uintptr_t>(p.mask) + (uint64_t)((mask_row(r) + k0) * esz)) & 15) == 0;
+        if (ok) {
+            pre_k0 = k0;
+            pre_end = k0 + nb / esz;
+            pre_rows = rows;
+            pre_pitch = nb;
+        }
+    }
 
     // Inputs and the split counters may come from the previous kernel of the
     // stream: wait for it to complete before the first global access.
@@ -239,11 +287,22 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
+        if (lane == 0 && pre_rows > 0) {
+            mbar_arrive_expect_tx(bar_mask, (uint32_t)pre_rows * pre_pitch);
+            for (int r = 0; r < pre_rows; ++r)
+                bulk_load(smem_u32(mpre) + r * pre_pitch,
+                          static_cast<const unsigned char*>(p.mask) + (mask_row(r) + pre_k0) * esz, pre_pitch,
+                          bar_mask);
+        }
         if (lane == 0 && n_slots > 0) {
             int t = 0;
             bool ok = true;
             for (; t < n_slots; ++t) {
                 const int slot = t % NSLOT;
+                if (C::INFLIGHT < NSLOT && t >= C::INFLIGHT &&
+                    !(ok = wait_phase(bar_full + (t - C::INFLIGHT) % NSLOT, ((t - C::INFLIGHT) / NSLOT) & 1,
+                                      kErrWaitTmaLoad, p.wait_limit_ns)))
+                    break;
                 if (t >= NSLOT &&
                     !(ok = wait_phase(bar_empty + slot, ((t / NSLOT) & 1) ^ 1, kErrWaitSlot, p.wait_limit_ns)))
                     break;
@@ -270,6 +329,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                 for (int x = (t > NSLOT ? t - NSLOT : 0); x < t; ++x)
                     wait_phase(bar_full + x % NSLOT, (x / NSLOT) & 1, kErrWaitTmaLoad, p.wait_limit_ns);
         }
+        if (lane == 0 && pre_rows > 0) wait_phase(bar_mask, 0, kErrWaitTmaLoad, p.wait_limit_ns);
     } else {
         // ------------------------------------------------------------ consumer warps
         // Q rows of this CTA (zero rows past the group and zero pad columns)
@@ -322,12 +382,21 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                     bool keep = row_ok[nt][rc] && j < p.Lk;
                     float add = 0.f;
                     if (keep && (p.mask_kind == 1 || p.mask_kind == 2)) {   // a mask tensor to read
-                        const int64_t moff =
-                            b * p.sm[0] + row_h[nt][rc] * p.sm[1] + row_i[nt][rc] * p.sm[2] + j * p.sm[3];
-                        if (p.mask_kind == 1)
-                            add = Elem<T>::to_float(reinterpret_cast<const T*>(p.mask)[moff]) * log2e;
-                        else
-                            keep = reinterpret_cast<const uint8_t*>(p.mask)[moff] != 0;
+                        if (j >= pre_k0 && j < pre_end) {
+                            const int rr = pre_rows == 1 ? 0 : nt * 8 + 2 * t4 + rc;
+                            const unsigned char* src = mpre + rr * pre_pitch + (j - pre_k0) * esz;
+                            if (p.mask_kind == 1)
+                                add = Elem<T>::to_float(*reinterpret_cast<const T*>(src)) * log2e;
+                            else
+                                keep = *src != 0;
+                        } else {
+                            const int64_t moff =
+                                b * p.sm[0] + row_h[nt][rc] * p.sm[1] + row_i[nt][rc] * p.sm[2] + j * p.sm[3];
+                            if (p.mask_kind == 1)
+                                add = Elem<T>::to_float(reinterpret_cast<const T*>(p.mask)[moff]) * log2e;
+                            else
+                                keep = reinterpret_cast<const uint8_t*>(p.mask)[moff] != 0;
+                        }
                     } else if (keep && p.mask_kind == 3) {
                         keep = j <= row_i[nt][rc] + p.Lk - p.Lq;
                     } else if (keep && p.mask_kind == 4) {
@@ -338,7 +407,11 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                     mf.keep[nt][c] = keep;
                 }
         };
-        const int n_items = n_slots * kNSUB;
+        // (if the mask copy never lands, the wait sets the error flag and this
+        // warp takes no sub-block: the producer's own waits then run out too)
+        const bool mask_ok =
+            pre_rows == 0 || __all_sync(0xffffffffu, wait_phase(bar_mask, 0, kErrWaitTmaLoad, p.wait_limit_ns));
+        const int n_items = mask_ok ? n_slots * kNSUB : 0;
         // one sub-block ahead where the registers allow (NT <= 2); with 32 rows
         // per CTA the values load right before the wait for the sub-block's data
         constexpr bool kAhead = NT <= 2;
@@ -349,102 +422,113 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         const uint32_t q_base = smem_u32(Qs);
         const int mi = lane >> 3;   // which 8x8 matrix this lane addresses in an x4 ldmatrix
 
-        for (int item = w; item < n_items; item += W) {
-            const int t = item / kNSUB, u = item % kNSUB;   // slot t, 16-key sub-block u
+        // Every consumer warp waits on every slot in order and releases it
+        // (bar_empty counts W arrivals), doing its own sub-blocks of the slot in
+        // between.  A parity wait is only unambiguous when the barrier has
+        // already completed the phase before the awaited one; a warp that
+        // waited only on the slots of its own sub-blocks could run two uses
+        // of a ring position ahead (with 7 warps and 3 slots of 2 sub-blocks,
+        // a warp's first sub-block already sits in a position's second use)
+        // and pass a wait on the wrong phase.
+        int item = w;   // this warp's next sub-block: w, w + W, ...
+        for (int t = 0; t < n_slots; ++t) {
             const int slot = t % NSLOT;
-            MaskFrag<NT> mcur;
-            if (kAhead) {
-                mcur = mnext;
-                // the next sub-block's mask values load while this one computes
-                if (item + W < n_items) load_mask(item + W, mnext);
-            } else {
-                load_mask(item, mcur);
-            }
             if (!__all_sync(0xffffffffu, wait_phase(bar_full + slot, (t / NSLOT) & 1, kErrWaitTmaLoad,
                                                     p.wait_limit_ns)))
                 break;
-            const uint32_t kbase = ring + slot * C::SLOT;
-            const uint32_t vbase = kbase + C::NBK * kChunk;
-            const int rsub = u * 16;   // first row of this sub-block inside the slot
-
-            // S^T[16 keys][8*NT rows] = K_blk . Q^T
-            float s[NT][4], s2[NT][4];   // even / odd K steps: two independent MMA chains
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) s[nt][c] = s2[nt][c] = 0.f;
-            {
-                const int arow = rsub + (mi & 1) * 8 + (lane & 7);
-                const uint32_t b_addr = q_base + (uint32_t)(((lane & 7) * C::QS + ((lane >> 3) & 1) * 8) * 2);
-#pragma unroll
-                for (int ks = 0; ks < C::DQKP / 16; ++ks) {
-                    uint32_t a0, a1, a2, a3;
-                    ldmatrix_x4(swz(kbase + (ks >> 2) * kChunk, arow, ((ks & 3) << 1) + (mi >> 1)), a0, a1, a2, a3);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        uint32_t b0, b1;
-                        ldmatrix_x2(b_addr + (uint32_t)(nt * 8 * C::QS * 2) + ks * 32, b0, b1);
-                        if (ks & 1)
-                            mma_16816<T>(s2[nt], a0, a1, a2, a3, b0, b1);
-                        else
-                            mma_16816<T>(s[nt], a0, a1, a2, a3, b0, b1);
-                    }
+            for (; item < n_items && item < (t + 1) * kNSUB; item += W) {
+                const int u = item - t * kNSUB;   // 16-key sub-block u of slot t
+                MaskFrag<NT> mcur;
+                if (kAhead) {
+                    mcur = mnext;
+                    // the next sub-block's mask values load while this one computes
+                    if (item + W < n_items) load_mask(item + W, mnext);
+                } else {
+                    load_mask(item, mcur);
                 }
+                const uint32_t kbase = ring + slot * C::SLOT;
+                const uint32_t vbase = kbase + C::NBK * kChunk;
+                const int rsub = u * 16;   // first row of this sub-block inside the slot
+
+                // S^T[16 keys][8*NT rows] = K_blk . Q^T
+                float s[NT][4], s2[NT][4];   // even / odd K steps: two independent MMA chains
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) s[nt][c] += s2[nt][c];
-            }
+                    for (int c = 0; c < 4; ++c) s[nt][c] = s2[nt][c] = 0.f;
+                {
+                    const int arow = rsub + (mi & 1) * 8 + (lane & 7);
+                    const uint32_t b_addr = q_base + (uint32_t)(((lane & 7) * C::QS + ((lane >> 3) & 1) * 8) * 2);
+#pragma unroll
+                    for (int ks = 0; ks < C::DQKP / 16; ++ks) {
+                        uint32_t a0, a1, a2, a3;
+                        ldmatrix_x4(swz(kbase + (ks >> 2) * kChunk, arow, ((ks & 3) << 1) + (mi >> 1)), a0, a1, a2, a3);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            uint32_t b0, b1;
+                            ldmatrix_x2(b_addr + (uint32_t)(nt * 8 * C::QS * 2) + ks * 32, b0, b1);
+                            if (ks & 1)
+                                mma_16816<T>(s2[nt], a0, a1, a2, a3, b0, b1);
+                            else
+                                mma_16816<T>(s[nt], a0, a1, a2, a3, b0, b1);
+                        }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) s[nt][c] += s2[nt][c];
+                }
 
-            // scale, mask, online softmax (log2 domain)
-            uint32_t pb[NT][2];
+                // scale, mask, online softmax (log2 domain)
+                uint32_t pb[NT][2];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                float bmax[2] = {-INFINITY, -INFINITY};
+                for (int nt = 0; nt < NT; ++nt) {
+                    float bmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float x = mcur.keep[nt][c] ? fmaf(s[nt][c], p.scale_log2, mcur.add[nt][c]) : -INFINITY;
-                    s[nt][c] = x;
-                    bmax[c & 1] = fmaxf(bmax[c & 1], x);
+                    for (int c = 0; c < 4; ++c) {
+                        const float x = mcur.keep[nt][c] ? fmaf(s[nt][c], p.scale_log2, mcur.add[nt][c]) : -INFINITY;
+                        s[nt][c] = x;
+                        bmax[c & 1] = fmaxf(bmax[c & 1], x);
+                    }
+                    float alpha[2], m_use[2];
+#pragma unroll
+                    for (int rc = 0; rc < 2; ++rc) {
+                        float v = bmax[rc];
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+                        const float m_new = fmaxf(m_run[nt][rc], v);
+                        m_use[rc] = (m_new == -INFINITY) ? 0.f : m_new;
+                        alpha[rc] = fast_exp2(m_run[nt][rc] - m_use[rc]);
+                        m_run[nt][rc] = m_new;
+                    }
+                    float pr[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) pr[c] = fast_exp2(s[nt][c] - m_use[c & 1]);
+                    l_run[nt][0] = l_run[nt][0] * alpha[0] + pr[0] + pr[2];
+                    l_run[nt][1] = l_run[nt][1] * alpha[1] + pr[1] + pr[3];
+#pragma unroll
+                    for (int mt = 0; mt < C::DVP / 16; ++mt) {
+                        o[mt][nt][0] *= alpha[0];
+                        o[mt][nt][1] *= alpha[1];
+                        o[mt][nt][2] *= alpha[0];
+                        o[mt][nt][3] *= alpha[1];
+                    }
+                    pb[nt][0] = movmatrix_trans(pack2<T>(pr[0], pr[1]));   // keys 0-7
+                    pb[nt][1] = movmatrix_trans(pack2<T>(pr[2], pr[3]));   // keys 8-15
                 }
-                float alpha[2], m_use[2];
-#pragma unroll
-                for (int rc = 0; rc < 2; ++rc) {
-                    float v = bmax[rc];
-                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-                    const float m_new = fmaxf(m_run[nt][rc], v);
-                    m_use[rc] = (m_new == -INFINITY) ? 0.f : m_new;
-                    alpha[rc] = fast_exp2(m_run[nt][rc] - m_use[rc]);
-                    m_run[nt][rc] = m_new;
-                }
-                float pr[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) pr[c] = fast_exp2(s[nt][c] - m_use[c & 1]);
-                l_run[nt][0] = l_run[nt][0] * alpha[0] + pr[0] + pr[2];
-                l_run[nt][1] = l_run[nt][1] * alpha[1] + pr[1] + pr[3];
-#pragma unroll
-                for (int mt = 0; mt < C::DVP / 16; ++mt) {
-                    o[mt][nt][0] *= alpha[0];
-                    o[mt][nt][1] *= alpha[1];
-                    o[mt][nt][2] *= alpha[0];
-                    o[mt][nt][3] *= alpha[1];
-                }
-                pb[nt][0] = movmatrix_trans(pack2<T>(pr[0], pr[1]));   // keys 0-7
-                pb[nt][1] = movmatrix_trans(pack2<T>(pr[2], pr[3]));   // keys 8-15
-            }
 
-            // O^T[DV][rows] += V^T . P^T
-            {
-                const int vrow = rsub + (mi >> 1) * 8 + (lane & 7);
+                // O^T[DV][rows] += V^T . P^T
+                {
+                    const int vrow = rsub + (mi >> 1) * 8 + (lane & 7);
 #pragma unroll
-                for (int mt = 0; mt < C::DVP / 16; ++mt) {
-                    uint32_t a0, a1, a2, a3;
-                    ldmatrix_x4_trans(swz(vbase + (mt >> 2) * kChunk, vrow, ((mt & 3) << 1) + (mi & 1)), a0, a1, a2,
-                                      a3);
+                    for (int mt = 0; mt < C::DVP / 16; ++mt) {
+                        uint32_t a0, a1, a2, a3;
+                        ldmatrix_x4_trans(swz(vbase + (mt >> 2) * kChunk, vrow, ((mt & 3) << 1) + (mi & 1)), a0, a1, a2,
+                                          a3);
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_16816<T>(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                        for (int nt = 0; nt < NT; ++nt) mma_16816<T>(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                    }
                 }
             }
             __syncwarp();
@@ -489,7 +573,6 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     }
     __syncthreads();
 
-    const int n_rows = (int)min((int64_t)C::ROWS, R - row0);   // real query rows of this CTA
     float* coef = reinterpret_cast<float*>(smem + C::OFF_COEF);   // [ROWS][W + 1]
     for (int r = tid; r < n_rows; r += C::THREADS) {            // per row: weights of the W warps, lse
         float mmax = -INFINITY;

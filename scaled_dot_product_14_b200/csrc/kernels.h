@@ -135,6 +135,8 @@ cudaError_t prefill_tc_launch(const AttnParams& p, int dtype, const LaunchPlan& 
 // api.cu: stores cudaGetErrorString(e) as this thread's sdpa_last_cuda_error
 // text, clears the runtime's pending error, and returns SDPA_ERR_CUDA.
 int record_cuda_error(cudaError_t e);
+// empties this thread's last-error text (every entry point does on entry)
+void clear_last_cuda_error();
 
 // ---- fp32 prefill on tcgen05 kind::tf32 with a three-term split: prefill_tf32.cu
 bool prefill_tf32_supported(int dtype, int64_t Dqk, int64_t Dv);

@@ -81,6 +81,7 @@ extern "C" int sdpa_forward_noalloc(const void* q, const void* k, const void* v,
                                     int64_t Hkv, int64_t Lq, int64_t Lk, int64_t Dqk, int64_t Dv,
                                     const int64_t strides[16], float scale, int mask_kind, const void* mask,
                                     const int64_t mask_strides[4], int dtype, void* stream_ptr) {
+    clear_last_cuda_error();
     // the same validation as sdpa_forward
     int path = SDPA_PATH_NONE;
     int st = sdpa_supported(B, Hq, Hkv, Lq, Lk, Dqk, Dv, strides, mask_kind, mask_strides, dtype, &path);

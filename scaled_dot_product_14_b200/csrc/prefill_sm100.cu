@@ -245,7 +245,6 @@ struct RowSoftmax {
         // values stay raw where possible and are scaled inside the exponent's FFMA
         float mul = sc;
         if (MASK == 1 || MASK == 2) {
-            mul = 1.f;
             // this tile's values: the vectors requested during the previous tile
             // (or now); they are applied first, and then the next tile's vectors
             // are requested, so one set is live at a time (an additive mask at
@@ -253,21 +252,51 @@ struct RowSoftmax {
             // the 128 scores would spill)
             if (mvec_kbase != kbase) fetch_mask(kbase);
             const bool vec = mvec_kbase == kbase;
-            const T* mt_row = mask_t + mrow + kbase * msm3;
-            const uint8_t* mb_row = mask_b + mrow + kbase * msm3;
+            if (__all_sync(0xffffffffu, vec) && !partial && (MASK == 1 || pos_scale)) {
+                // every key of the tile visible and the values in registers: no
+                // branch per key
+                if (MASK == 2) {
+                    // boolean: hidden keys become -inf on the raw score; the scale
+                    // stays in the exponent's multiplier (positive scale)
+                    const uint32_t* w = reinterpret_cast<const uint32_t*>(mvec);
 #pragma unroll
-            for (int c = 0; c < NK; ++c) {
-                float x = __uint_as_float(sr[c]) * sc;
-                bool keep = c < vis && c >= lo;
-                if (MASK == 1 && keep) {
-                    const T mv = vec ? reinterpret_cast<const T*>(mvec)[c] : mt_row[(int64_t)c * msm3];
-                    x += Elem<T>::to_float(mv) * log2e;
+                    for (int g = 0; g < NK / 4; ++g) {
+                        const uint32_t keepb = __vcmpne4(w[g], 0u);   // 0xff per visible key
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t m = (uint32_t)((int32_t)(keepb << (24 - 8 * e)) >> 31);
+                            sr[4 * g + e] = (sr[4 * g + e] & m) | (0xff800000u & ~m);
+                        }
+                    }
+                } else {
+                    // additive: s * scale + m in natural-log units; log2(e) moves
+                    // into the exponent's multiplier
+                    mul = log2e;
+                    const float scn = sc / log2e;
+                    const T* mv = reinterpret_cast<const T*>(mvec);
+#pragma unroll
+                    for (int c = 0; c < NK; ++c)
+                        sr[c] = __float_as_uint(fmaf(__uint_as_float(sr[c]), scn, Elem<T>::to_float(mv[c])));
                 }
-                if (MASK == 2 && keep) {
-                    const uint8_t mb = vec ? reinterpret_cast<const uint8_t*>(mvec)[c] : mb_row[(int64_t)c * msm3];
-                    keep = mb != 0;
+            } else {
+                mul = 1.f;
+                const T* mt_row = mask_t + mrow + kbase * msm3;
+                const uint8_t* mb_row = mask_b + mrow + kbase * msm3;
+#pragma unroll
+                for (int c = 0; c < NK; ++c) {
+                    float x = __uint_as_float(sr[c]) * sc;
+                    bool keep = c < vis && c >= lo;
+                    if (MASK == 1 && keep) {
+                        const T mv = vec ? reinterpret_cast<const T*>(mvec)[c] : mt_row[(int64_t)c * msm3];
+                        x += Elem<T>::to_float(mv) * log2e;
+                    }
+                    if (MASK == 2 && keep) {
+                        const uint8_t mb =
+                            vec ? reinterpret_cast<const uint8_t*>(mvec)[c] : mb_row[(int64_t)c * msm3];
+                        keep = mb != 0;
+                    }
+                    sr[c] = __float_as_uint(keep ? x : -INFINITY);
                 }
-                sr[c] = __float_as_uint(keep ? x : -INFINITY);
             }
             fetch_mask(kbase + NK);
         } else if (!pos_scale) {

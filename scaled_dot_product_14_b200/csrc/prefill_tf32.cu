@@ -109,16 +109,19 @@ __device__ __forceinline__ void split_tf32(unsigned char* hi, unsigned char* lo,
 // V(j) as loaded ([key][dv] in NV chunks of 64 keys x 32 dv, 128-byte
 // swizzled rows) -> V^T hi and lo as K-major tiles for the P V MMA: for each
 // chunk of 32 keys, DVP rows (dv) of 128 bytes (32 keys), 128-byte swizzled.
-// Rows dv >= NV * 32 do not exist (DVP <= NV * 32).  By `n` threads.
+// Rows dv >= NV * 32 do not exist (DVP <= NV * 32).  By `n` threads, n a
+// multiple of 32: the 32 lanes of a warp take 32 consecutive keys of one
+// 16-byte unit, so each quarter-warp reads 8 distinct swizzled units and each
+// transposed store of the warp hits 32 distinct banks.
 template <int NV, int DVP>
 __device__ __forceinline__ void split_transpose_v(const unsigned char* raw, unsigned char* th, unsigned char* tl,
                                                   int t, int n) {
     constexpr int VT_CHUNK = DVP * 128;
-    for (int i = t; i < NV * 64 * 8; i += n) {   // 16-byte units: chunk c, key r, logical unit u
-        const int c = i / (64 * 8), r = (i / 8) % 64, u = i % 8;
+    for (int i = t; i < NV * 64 * 8; i += n) {   // 16-byte units: chunk c, key chunk kc, logical unit u, key kk
+        const int kk = i & 31, u = (i >> 5) & 7, kc = (i >> 8) & 1, c = i >> 9;
+        const int r = kc * 32 + kk;
         const uint4 x = *reinterpret_cast<const uint4*>(raw + c * kKChunk + r * 128 + ((u ^ (r & 7)) << 4));
         const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
-        const int kc = r >> 5, kk = r & 31;
 #pragma unroll
         for (int e4 = 0; e4 < 4; ++e4) {
             const int e = c * 32 + u * 4 + e4;   // dv row of V^T

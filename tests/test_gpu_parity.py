@@ -113,6 +113,29 @@ def test_decode_d512_gqa8(kL, mask):
     run_and_check(c, label=f"decode d512 kL={kL} {mask}")
 
 
+@pytest.mark.parametrize("splits", [1, 4, 16, "one wave"])
+@pytest.mark.parametrize("D,Hkv", [(512, 4), (256, 8), (64, 8)])
+@pytest.mark.parametrize("mask", ["none", "decode_additive"])
+def test_decode_ring_reuse(monkeypatch, splits, D, Hkv, mask):
+    """Few splits give each CTA many key slots, so every ring position of the
+    decode kernel is reused many times (at D = 512 the ring has 3 positions of
+    2 sub-blocks for 7 consumer warps, so a warp's first sub-block can already
+    sit in a position's second use).  Repeated calls: a race would show as a
+    mismatch in some of them."""
+    if splits == "one wave":   # as many splits as fill the SMs (the default plan's count)
+        splits = torch.cuda.get_device_properties(0).multi_processor_count // Hkv
+    monkeypatch.setenv("SDPA_DECODE_SPLITS", str(splits))
+    c = I.make_case(1003, 1, 32, Hkv, 1, 4096, D, dtype=I.BF16, mask=mask)
+    g = GpuCase(c)
+    ref = oracle_rows(c).reshape(-1, D)
+    for _ in range(3):
+        assert g.run() == 0
+        got = g.output().reshape(-1, D)
+        err = np.abs(got - ref)
+        assert err.max() <= 2e-2 and err.mean() <= 2e-3, (splits, D, mask, float(err.max()), float(err.mean()))
+    assert S.sdpa_check_device_error() == (0, 0)
+
+
 def test_prefill_d512_causal_4096():
     c = I.make_case(1002, 1, 32, 4, 4096, 4096, 512, dtype=I.BF16, mask="causal")
     rows = I.sample_rows(1002, 1, 32, 4096, 96)

@@ -702,10 +702,18 @@ Shape shape_of() {
     X(256, 256, 7, 6, 32)   \
     X(512, 512, 7, 3, 32)
 
+// Head dim 512 has a second variant with 16-key slots (a ring of 6): when the
+// CTAs of a call hold more slots than the 3-slot ring, its deeper ring keeps
+// more loads queued behind the in-order slot releases (measured at kL = 4096:
+// 14.4 us against 16.6); with one or two slots per CTA the 32-key variant is
+// faster (10.7 us against 11.9 at kL = 1024).
+#define SDPA_DECODE_D512_DEEP 7, 6, 16
+
 constexpr int nt_cap(int dv) { return dv >= 512 ? 1 : (dv >= 256 ? 2 : 4); }
 constexpr int nt_fix(int want, int dv) { return want < nt_cap(dv) ? want : nt_cap(dv); }
 
-Shape pick_shape(int64_t Dqk, int64_t Dv, int64_t rows) {
+Shape pick_shape(int64_t Dqk, int64_t Dv, int64_t rows, bool deep = false) {
+    if (deep && Dqk == 512 && Dv == 512) return shape_of<512, 512, 1, SDPA_DECODE_D512_DEEP>();
     const int need = (int)((rows + 7) / 8);
     int nt = 1;
     while (nt < need && nt < nt_cap((int)Dv)) nt *= 2;
@@ -757,6 +765,8 @@ template <typename T>
 cudaError_t launch_typed(const DecParams& dp, const CUtensorMap& mk, const CUtensorMap& mv, const LaunchPlan& plan,
                          cudaStream_t s) {
     const int nt = plan.aux;
+    if (plan.slot_keys == 16 && dp.p.Dqk == 512 && dp.p.Dv == 512)
+        return launch_one<T, 512, 512, 1, SDPA_DECODE_D512_DEEP>(dp, mk, mv, plan, s);
     switch (dp.p.Dqk * 1000 + dp.p.Dv) {
 #define SDPA_DECODE_LAUNCH(DQ, DVV, W, NS, SK)                                                       \
     case DQ * 1000 + DVV:                                                                            \
@@ -786,8 +796,15 @@ LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev
     (void)dtype;
     LaunchPlan plan{};
     const int64_t rows = (int64_t)p.group * p.Lq;
-    const Shape sh = pick_shape(p.Dqk, p.Dv, rows);
+    Shape sh = pick_shape(p.Dqk, p.Dv, rows);
     if (sh.smem == 0 || rows <= 0 || p.B <= 0 || p.Hkv <= 0) return plan;
+    {   // more slots per CTA than the ring holds: the deeper-ring variant (head dim 512)
+        const Shape deep = pick_shape(p.Dqk, p.Dv, rows, true);
+        const int64_t groups0 = p.B * p.Hkv * ((rows + 8 * sh.nt - 1) / (8 * sh.nt));
+        const int64_t splits0 = groups0 < dev.sm_count ? dev.sm_count / groups0 : 1;
+        const int64_t slots0 = (p.Lk + sh.sk - 1) / sh.sk;
+        if (deep.sk != sh.sk && (slots0 + splits0 - 1) / splits0 > sh.nslot) sh = deep;
+    }
     const int64_t RG = (rows + 8 * sh.nt - 1) / (8 * sh.nt);
     // slots of sh.sk keys per group that some row may see (a sliding window
     // covers at most window + Lq - 1 keys, which may straddle one more slot)
@@ -831,6 +848,7 @@ LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev
     plan.keys_per_split = ((nsl + lo - 1) / lo) * sh.sk;   // the largest split (informational)
     plan.variant = (int)RG;
     plan.aux = sh.nt;
+    plan.slot_keys = sh.sk;
     return plan;
 }
 
@@ -851,7 +869,7 @@ cudaError_t decode_mma_launch(const AttnParams& p, int dtype, const LaunchPlan& 
     dp.extra = plan.split_extra;
     dp.s_max = plan.splits;
     dp.counters = counters;
-    const int sk = pick_shape(p.Dqk, p.Dv, (int64_t)p.group * p.Lq).sk;
+    const int sk = plan.slot_keys;
     CUtensorMap mk, mv;
     const bool ok_k = p.Dqk % 64 == 0
                           ? make_tensor_map_rows(&mk, &dp.k_ax, p.k, dtype, p.Dqk, p.Lk, p.Hkv, p.B, p.sk, sk)

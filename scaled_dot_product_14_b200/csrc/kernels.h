@@ -76,6 +76,7 @@ struct LaunchPlan {
     // split_lo (splits = the larger, the row stride of the partials)
     int split_lo;
     int split_extra;
+    int slot_keys;        // decode: keys per ring slot of the chosen variant
 };
 
 struct DeviceInfo {

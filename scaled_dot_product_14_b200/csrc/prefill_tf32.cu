@@ -19,11 +19,11 @@
 //               its own) and V^T read K-major from shared memory (every tf32
 //               operand here is K-major: that is the form the 128-byte swizzle
 //               of the tiles describes for 32-bit elements);
-//   warps 2-3   split each landed tile: Q and K in place (hi over the raw
+//   warps 2-7   split each landed tile: Q and K in place (hi over the raw
 //               values, lo into a buffer of the same swizzled layout, so the
 //               split is element-wise and both copies take one descriptor
 //               form), V transposed into K-major V^T hi and lo tiles;
-//   warps 4-7   softmax: thread t owns query row t (TMEM lane t), fp32 running
+//   warps 8-11  softmax: thread t owns query row t (TMEM lane t), fp32 running
 //               max / sum in the log2 domain, masks (none, additive, boolean,
 //               causal, sliding window), P split into hi / lo and written to
 //               TMEM, O rescaled in TMEM only when the row maximum grew by more
@@ -46,7 +46,8 @@ constexpr int kBMf = 128;                 // query rows per CTA (UMMA M)
 constexpr int kBNf = 64;                  // keys per tile (UMMA N of S, K of P V)
 constexpr int kQChunk = kBMf * 128;       // 128 rows x 32 fp32
 constexpr int kKChunk = kBNf * 128;       // 64 rows x 32 fp32
-constexpr int kThreadsF = 256;            // 8 warps
+constexpr int kThreadsF = 384;            // 12 warps
+constexpr int kSplitThreads = 192;        // warps 2-7 split each landed tile into hi / lo
 constexpr float kRescaleThresholdF = 8.0f;
 
 __host__ __device__ constexpr int cdivf(int a, int b) { return (a + b - 1) / b; }
@@ -224,13 +225,13 @@ __global__ void __launch_bounds__(kThreadsF, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q_full, 1);
-        mbar_init(bar_q_conv, 64);
+        mbar_init(bar_q_conv, kSplitThreads);
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(bar_k_full + s, 1);
-            mbar_init(bar_k_conv + s, 64);
+            mbar_init(bar_k_conv + s, kSplitThreads);
             mbar_init(bar_k_empty + s, 1);
             mbar_init(bar_v_full + s, 1);
-            mbar_init(bar_v_conv + s, 64);
+            mbar_init(bar_v_conv + s, kSplitThreads);
             mbar_init(bar_v_empty + s, 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -345,13 +346,13 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             umma_commit(bar_drain);
             wait_phase(bar_drain, 0, kErrWaitMma);
         }
-    } else if (warp < 4) {
+    } else if (warp < 2 + kSplitThreads / 32) {
         // ------------------------------------------------------------ hi / lo split
         const int t = threadIdx.x - 64;
         if (n_tiles > 0) {
             bool ok = wait_phase(bar_q_full, 0, kErrWaitTmaLoad);
             if (ok) {
-                split_tf32(smem + C::OFF_QH, smem + C::OFF_QL, C::Q_BYTES, t, 64);
+                split_tf32(smem + C::OFF_QH, smem + C::OFF_QL, C::Q_BYTES, t, kSplitThreads);
                 fence_proxy_async();   // the tensor core reads them through the async proxy
                 mbar_arrive(bar_q_conv);
             }
@@ -359,18 +360,18 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                 const int st = j % NSTAGE;
                 const uint32_t par = (j / NSTAGE) & 1;
                 if (!(ok = wait_phase(bar_k_full + st, par, kErrWaitTmaLoad))) break;
-                split_tf32(smem + kh(st), smem + kl(st), C::K_BYTES, t, 64);
+                split_tf32(smem + kh(st), smem + kl(st), C::K_BYTES, t, kSplitThreads);
                 fence_proxy_async();
                 mbar_arrive(bar_k_conv + st);
                 if (!(ok = wait_phase(bar_v_full + st, par, kErrWaitTmaLoad))) break;
-                split_transpose_v<C::NV, C::DVP>(smem + vraw(st), smem + vth(st), smem + vtl(st), t, 64);
+                split_transpose_v<C::NV, C::DVP>(smem + vraw(st), smem + vth(st), smem + vtl(st), t, kSplitThreads);
                 fence_proxy_async();
                 mbar_arrive(bar_v_conv + st);
             }
         }
     } else {
         // ------------------------------------------------------------ softmax / epilogue
-        const int quad = warp & 3;   // warps 4..7 -> TMEM lane quadrants 0..3
+        const int quad = warp & 3;   // warps 8..11 -> TMEM lane quadrants 0..3
         const int r = quad * 32 + lane;
         const int64_t i = q0 + r;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;

@@ -264,7 +264,8 @@ struct RowSoftmax {
                         const uint32_t keepb = __vcmpne4(w[g], 0u);   // 0xff per visible key
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const uint32_t m = (uint32_t)((int32_t)(keepb << (24 - 8 * e)) >> 31);
+                            // byte e's sign replicated over the word (byte-permute selector 8 + e)
+                            const uint32_t m = __byte_perm(keepb, 0u, (8u + e) * 0x1111u);
                             sr[4 * g + e] = (sr[4 * g + e] & m) | (0xff800000u & ~m);
                         }
                     }

@@ -439,3 +439,23 @@ def test_sliding_window_abi_rules():
                             None, c.dtype) == (0, S.SDPA_PATH_PREFILL)
     assert S.sdpa_forward_window(*args, 5, c.dtype, s) == 0
     torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- many heads, GQA, ragged (head dims 64-96)
+# The 96-key-tile kernel on grids of 16, 160 and 240 two-tile CTAs (on 148 SMs:
+# under one wave, one wave and a little, one and a half waves), with GQA
+# groups of 1, 3 and 8, ragged query and key lengths, every mask kind; all rows
+# are checked.
+@pytest.mark.parametrize("D", [64, 72, 96])
+@pytest.mark.parametrize("dtype", [I.BF16, I.F16])
+@pytest.mark.parametrize("shape", [
+    dict(Hq=4, Hkv=4, Lq=1000, Lk=1000),
+    dict(Hq=80, Hkv=10, Lq=500, Lk=509),
+    dict(Hq=120, Hkv=40, Lq=512, Lk=384),
+])
+@pytest.mark.parametrize("mask", ["none", "bool", "additive", "causal"])
+def test_prefill_many_heads_ragged(D, dtype, shape, mask):
+    seed = 5100 + D + 7 * shape["Hq"] + (mask == "bool") * 3 + (mask == "additive") * 5 + (mask == "causal") * 11
+    c = I.make_case(seed, 1, shape["Hq"], shape["Hkv"], shape["Lq"], shape["Lk"], D, dtype=dtype, mask=mask,
+                    layout="blhd")
+    run_and_check(c, None, label=f"many heads D={D} {shape} {mask}")

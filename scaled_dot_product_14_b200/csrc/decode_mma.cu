@@ -786,11 +786,9 @@ bool decode_mma_supported(int dtype, int64_t Dqk, int64_t Dv) {
 }
 
 // Work split.  A (batch, KV head, row group) is a group; its slots of keys are
-// split across CTAs so that the grid has one CTA per SM (the kernel takes most
-// of the shared memory): with `groups` groups on `sm` SMs, the first sm % groups
-// groups take sm / groups + 1 splits and the others sm / groups, each split at
-// most one slot short of the others.  More groups than SMs: one CTA per group,
-// in waves.  A head-dim pair this kernel does not cover gets an empty grid,
+// split across CTAs, at most one CTA per SM (the kernel takes most of the
+// shared memory), every group the same number of splits, each split at most one
+// slot short of the others.  More groups than SMs: one CTA per group, in waves.  A head-dim pair this kernel does not cover gets an empty grid,
 // which every caller refuses.
 LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev) {
     (void)dtype;
@@ -817,16 +815,17 @@ LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev
     const int64_t groups = p.B * p.Hkv * RG;
     int64_t lo = 1, extra = 0;
     if (groups < dev.sm_count) {
-        lo = dev.sm_count / groups;
-        extra = dev.sm_count % groups;
-        if (lo >= nsl) {   // every split gets at least one slot
-            lo = nsl > 0 ? nsl : 1;
-            extra = 0;
-        }
-        if (lo + (extra > 0) > kMaxSplits - 1) {
-            lo = kMaxSplits - 1;
-            extra = 0;
-        }
+        // Every group takes the same number of splits: the slowest split sets
+        // the launch time, so a group given one split more than the others
+        // gains nothing.  The cap is the SMs' share per group, and half the
+        // slots (each split adds a partial to merge, and a one-slot split is
+        // mostly fixed cost).  Under the cap, the fewest splits that reach the
+        // smallest largest share of slots.
+        int64_t cap = dev.sm_count / groups;
+        if (cap > nsl / 2) cap = nsl / 2 > 1 ? nsl / 2 : 1;
+        if (cap > kMaxSplits - 1) cap = kMaxSplits - 1;
+        const int64_t m = (nsl + cap - 1) / cap;   // slots of the largest split
+        lo = m > 0 ? (nsl + m - 1) / m : 1;
     }
     // debugging override: the same number of splits for every group; a grid
     // that cannot be resident at once makes the cooperative launch fail

@@ -122,7 +122,7 @@ def test_decode_ring_reuse(monkeypatch, splits, D, Hkv, mask):
     2 sub-blocks for 7 consumer warps, so a warp's first sub-block can already
     sit in a position's second use).  Repeated calls: a race would show as a
     mismatch in some of them."""
-    if splits == "one wave":   # as many splits as fill the SMs (the default plan's count)
+    if splits == "one wave":   # as many splits as fill the SMs
         splits = torch.cuda.get_device_properties(0).multi_processor_count // Hkv
     monkeypatch.setenv("SDPA_DECODE_SPLITS", str(splits))
     c = I.make_case(1003, 1, 32, Hkv, 1, 4096, D, dtype=I.BF16, mask=mask)

@@ -459,3 +459,18 @@ def test_prefill_many_heads_ragged(D, dtype, shape, mask):
     c = I.make_case(seed, 1, shape["Hq"], shape["Hkv"], shape["Lq"], shape["Lk"], D, dtype=dtype, mask=mask,
                     layout="blhd")
     run_and_check(c, None, label=f"many heads D={D} {shape} {mask}")
+
+
+# ---------------------------------------------------------------- decode split plan
+# The decode plan gives every (batch, KV head, row group) the same split count:
+# at most the SMs' share per group and half the key slots, then the fewest
+# splits that reach the smallest largest share.  These shapes land on each
+# branch (one split; capped by the slots; capped by the SMs; more groups than
+# SMs, in waves) with ragged key counts; all rows against the oracle.
+@pytest.mark.parametrize("D", [64, 256, 512])
+@pytest.mark.parametrize("B,Hkv,group", [(1, 1, 4), (1, 8, 4), (2, 40, 2), (4, 48, 1)])
+@pytest.mark.parametrize("Lk", [1, 33, 95, 200, 1000, 5000])
+def test_decode_split_plan(D, B, Hkv, group, Lk):
+    mask = "decode_additive" if Lk % 2 == 1 else "none"
+    c = I.make_case(6100 + D + Hkv + Lk, B, Hkv * group, Hkv, 1, Lk, D, dtype=I.BF16, mask=mask)
+    run_and_check(c, None, label=f"decode split plan D={D} B={B} Hkv={Hkv} G={group} Lk={Lk}")

@@ -796,6 +796,7 @@ LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev
     const int64_t rows = (int64_t)p.group * p.Lq;
     Shape sh = pick_shape(p.Dqk, p.Dv, rows);
     if (sh.smem == 0 || rows <= 0 || p.B <= 0 || p.Hkv <= 0) return plan;
+    const int base_sk = sh.sk;   // the split count is chosen in slots of this size
     {   // more slots per CTA than the ring holds: the deeper-ring variant (head dim 512)
         const Shape deep = pick_shape(p.Dqk, p.Dv, rows, true);
         const int64_t groups0 = p.B * p.Hkv * ((rows + 8 * sh.nt - 1) / (8 * sh.nt));
@@ -804,14 +805,21 @@ LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev
         if (deep.sk != sh.sk && (slots0 + splits0 - 1) / splits0 > sh.nslot) sh = deep;
     }
     const int64_t RG = (rows + 8 * sh.nt - 1) / (8 * sh.nt);
-    // slots of sh.sk keys per group that some row may see (a sliding window
+    // slots of sk keys per group that some row may see (a sliding window
     // covers at most window + Lq - 1 keys, which may straddle one more slot)
-    int64_t nsl = (p.Lk + sh.sk - 1) / sh.sk;
-    if (p.mask_kind == 4) {
-        const int64_t vis = p.window + p.Lq - 1 < p.Lk ? p.window + p.Lq - 1 : p.Lk;
-        const int64_t nsl_vis = (vis + sh.sk - 1) / sh.sk + 1;
-        if (nsl_vis < nsl) nsl = nsl_vis;
-    }
+    auto visible_slots = [&](int64_t sk) {
+        int64_t n = (p.Lk + sk - 1) / sk;
+        if (p.mask_kind == 4) {
+            const int64_t vis = p.window + p.Lq - 1 < p.Lk ? p.window + p.Lq - 1 : p.Lk;
+            const int64_t n_vis = (vis + sk - 1) / sk + 1;
+            if (n_vis < n) n = n_vis;
+        }
+        return n;
+    };
+    const int64_t nsl = visible_slots(sh.sk);
+    // the split count is chosen on the head dim's base slot, so that the
+    // deeper ring (half-size slots) changes only how a split streams its keys
+    const int64_t nsb = visible_slots(base_sk);
     const int64_t groups = p.B * p.Hkv * RG;
     int64_t lo = 1, extra = 0;
     if (groups < dev.sm_count) {
@@ -822,10 +830,10 @@ LaunchPlan decode_mma_plan(const AttnParams& p, int dtype, const DeviceInfo& dev
         // mostly fixed cost).  Under the cap, the fewest splits that reach the
         // smallest largest share of slots.
         int64_t cap = dev.sm_count / groups;
-        if (cap > nsl / 2) cap = nsl / 2 > 1 ? nsl / 2 : 1;
+        if (cap > nsb / 2) cap = nsb / 2 > 1 ? nsb / 2 : 1;
         if (cap > kMaxSplits - 1) cap = kMaxSplits - 1;
-        const int64_t m = (nsl + cap - 1) / cap;   // slots of the largest split
-        lo = m > 0 ? (nsl + m - 1) / m : 1;
+        const int64_t m = (nsb + cap - 1) / cap;   // base slots of the largest split
+        lo = m > 0 ? (nsb + m - 1) / m : 1;
     }
     // debugging override: the same number of splits for every group; a grid
     // that cannot be resident at once makes the cooperative launch fail

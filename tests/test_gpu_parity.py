@@ -474,3 +474,24 @@ def test_decode_split_plan(D, B, Hkv, group, Lk):
     mask = "decode_additive" if Lk % 2 == 1 else "none"
     c = I.make_case(6100 + D + Hkv + Lk, B, Hkv * group, Hkv, 1, Lk, D, dtype=I.BF16, mask=mask)
     run_and_check(c, None, label=f"decode split plan D={D} B={B} Hkv={Hkv} G={group} Lk={Lk}")
+
+
+# The split counts the decode plan picks for the measured decode shapes on a
+# 148-SM B200 (read from the SDPA_LOG line of each call): every KV head gets the
+# same count, the one the split-count sweep found fastest or within 1 % of it.
+@pytest.mark.parametrize("D,Hkv,Lk,splits", [(256, 8, 4096, 16), (256, 8, 1024, 16),
+                                             (512, 4, 1024, 16), (512, 4, 4096, 32)])
+def test_decode_plan_split_counts(monkeypatch, capfd, D, Hkv, Lk, splits):
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("split counts pinned for 148 SMs")
+    monkeypatch.setenv("SDPA_LOG", "1")
+    c = I.make_case(6400 + D + Lk, 1, 32, Hkv, 1, Lk, D, dtype=I.BF16, mask="none")
+    rows = I.sample_rows(6400 + D, 1, 32, 1, 8)
+    run_and_check(c, rows, label=f"plan D={D} Lk={Lk}")
+    err = capfd.readouterr().err
+    lines = [l for l in err.splitlines() if l.startswith("[sdpa]") and f"Lk={Lk} Dqk={D}" in l]
+    assert lines, err
+    import re
+    m = re.search(r"grid=\((\d+),1,1\).*splits=(\d+)", lines[-1])
+    assert m, lines[-1]
+    assert int(m.group(2)) == splits and int(m.group(1)) == Hkv * splits, lines[-1]

@@ -227,11 +227,12 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     const int n_rows = (int)min((int64_t)C::ROWS, R - row0);   // real query rows of this CTA
 
     // ---- additive / boolean mask values of this CTA's keys go to shared memory
-    // up front, one bulk copy per distinct mask row issued before the first K/V
-    // slot, when each row's run is contiguous and 16-byte aligned and all of
-    // them fit: loads issued later would queue behind the CTA's K/V stream.
-    // Keys [pre_k0, pre_end) are then read from shared memory (the ragged
-    // last bytes of the run, if any, from global memory).
+    // up front, one bulk copy per distinct mask row issued right behind the
+    // first K/V slot (ahead of it, it delayed that slot; after several slots,
+    // it would queue behind the CTA's K/V stream), when each row's run is
+    // contiguous and 16-byte aligned and all of them fit.  Keys [pre_k0,
+    // pre_end) are then read from shared memory (the ragged last bytes of the
+    // run, if any, from global memory).
     const int64_t esz = p.mask_kind == 1 ? (int64_t)sizeof(T) : 1;
     auto mask_row = [&](int r) -> int64_t {   // element offset of CTA row r's mask row
         const int64_t gr = row0 + r;
@@ -287,13 +288,6 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0 && pre_rows > 0) {
-            mbar_arrive_expect_tx(bar_mask, (uint32_t)pre_rows * pre_pitch);
-            for (int r = 0; r < pre_rows; ++r)
-                bulk_load(smem_u32(mpre) + r * pre_pitch,
-                          static_cast<const unsigned char*>(p.mask) + (mask_row(r) + pre_k0) * esz, pre_pitch,
-                          bar_mask);
-        }
         if (lane == 0 && n_slots > 0) {
             int t = 0;
             bool ok = true;
@@ -324,6 +318,15 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                     for (int c = 0; c < C::NBV; ++c)
                         tma_load(base + (C::NBK + c) * kChunk, &tmV, bar_full + slot, dp.v_ax, c * 64, key0, hkv,
                                  b);
+                // the mask values right behind the first slot (pre_rows > 0 implies
+                // n_slots > 0, and slot 0 is issued without a wait, so this always runs)
+                if (t == 0 && pre_rows > 0) {
+                    mbar_arrive_expect_tx(bar_mask, (uint32_t)pre_rows * pre_pitch);
+                    for (int r = 0; r < pre_rows; ++r)
+                        bulk_load(smem_u32(mpre) + r * pre_pitch,
+                                  static_cast<const unsigned char*>(p.mask) + (mask_row(r) + pre_k0) * esz, pre_pitch,
+                                  bar_mask);
+                }
             }
             if (!ok)   // every issued load must land before shared memory is reused or released
                 for (int x = (t > NSLOT ? t - NSLOT : 0); x < t; ++x)
